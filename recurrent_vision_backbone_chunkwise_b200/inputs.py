@@ -1,0 +1,79 @@
+"""Seeded synthetic inputs shared by the oracle-side tests and the CUDA path.
+
+This module draws random numbers and nothing else: it holds none of the
+method's arithmetic, imports neither the oracle nor the CUDA binding, and is
+the only code the two sides have in common.
+
+Recipe (stands in for the GLA inputs of GTR's backbone at the 640x640
+detection, 1024x1024 segmentation and 2048x2048 high-resolution patch grids,
+stride-16 patch tokens; "GTR: Gated Token Recurrence for Efficient Dense
+Prediction", x-techcon article, sections 架构 and 算子):
+
+* one CPU ``torch.Generator`` seeded with ``seed``;
+* draw order q, k, v, then the gate pre-activations, each ``randn`` in fp32;
+* k is divided by sqrt(d_k) (no scale is applied inside the operator);
+* gates: ``logsigmoid(x) / 16`` ("normal") or ``logsigmoid(x + 2)``
+  ("stress": near-1 gates, long memory); every log-gate is finite and <= 0;
+* q, k, v are then cast to the I/O dtype; log_alpha stays fp32.
+
+Tensors come back on the CPU with layout [B, H, grid_h, grid_w, d].
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+
+import torch
+
+DTYPES = {"f16": torch.float16, "bf16": torch.bfloat16, "f32": torch.float32}
+
+
+@dataclass(frozen=True)
+class Shape:
+    B: int
+    H: int
+    grid_h: int
+    grid_w: int
+    d_k: int
+    d_v: int
+
+    @property
+    def tokens(self) -> int:
+        return self.grid_h * self.grid_w
+
+
+def make_inputs(shape: Shape, dtype: str = "f16", seed: int = 0, gates: str = "normal"):
+    """Return (q, k, v, log_alpha) CPU tensors for ``shape``."""
+    if dtype not in DTYPES:
+        raise ValueError(f"dtype must be one of {sorted(DTYPES)}")
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    s = shape
+    qk_shape = (s.B, s.H, s.grid_h, s.grid_w, s.d_k)
+    v_shape = (s.B, s.H, s.grid_h, s.grid_w, s.d_v)
+    q = torch.randn(qk_shape, generator=g, dtype=torch.float32)
+    k = torch.randn(qk_shape, generator=g, dtype=torch.float32)
+    v = torch.randn(v_shape, generator=g, dtype=torch.float32)
+    x = torch.randn(qk_shape, generator=g, dtype=torch.float32)
+    k = k / math.sqrt(s.d_k)
+    if gates == "normal":
+        log_alpha = torch.nn.functional.logsigmoid(x) / 16.0
+    elif gates == "stress":
+        log_alpha = torch.nn.functional.logsigmoid(x + 2.0)
+    else:
+        raise ValueError("gates must be 'normal' or 'stress'")
+    dt = DTYPES[dtype]
+    return (q.to(dt).contiguous(), k.to(dt).contiguous(), v.to(dt).contiguous(),
+            log_alpha.contiguous())
+
+
+# The workloads named for this operator: (name, Shape, dtype, directions).
+CONFIGS = {
+    "tiny": (Shape(1, 2, 16, 16, 64, 64), "f32"),
+    "640_b1": (Shape(1, 6, 40, 40, 64, 64), "f16"),
+    "640_b8": (Shape(8, 12, 40, 40, 64, 64), "f16"),
+    "1024_b1": (Shape(1, 12, 64, 64, 64, 64), "f16"),
+    "1024_b4": (Shape(4, 12, 64, 64, 64, 64), "f16"),
+    "16k_d64": (Shape(1, 12, 128, 128, 64, 64), "f16"),
+    "16k_d128": (Shape(1, 12, 128, 128, 128, 128), "f16"),
+}
