@@ -1,0 +1,369 @@
+#!/usr/bin/env python
+"""Throughput of the chunkwise key-gated linear attention forward pass.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--config 640_b1] [--no-graph]
+
+One step = the four scan directions (L->R, R->L, T->B, B->T, one call each,
+as four consecutive GTR layers would issue them) over one batch of synthetic
+input of the chosen workload.  Default workload: the 640x640 detection shape,
+B=1, H=6, 40x40 patch grid (1600 tokens), d_k = d_v = 64, fp16.
+
+Timing: W untimed warm-up steps, then exactly K steps bracketed by a barrier
+and a device synchronisation on both sides, timed with CUDA events on the
+launching stream; the timed steps are replayed from one CUDA graph (per-call
+events inside it give the per-launch durations).  Inputs rotate over enough
+separate buffers that each step reads data that is not in L2.  Under torchrun
+every rank runs its own replica (B*H planes are independent: no collective on
+the data path) and rank 0 prints one JSON line with the max time over ranks.
+
+--impl reference times the fp64 CPU oracle (the only other place this file
+runs it) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from recurrent_vision_backbone_chunkwise_b200.inputs import CONFIGS, make_inputs  # noqa: E402
+
+METRIC = "GLA fwd tokens/s and µs at 1600/4096/16384 tokens; % of roofline (HBM or TC)"
+L2_BYTES = 126 * 1024 * 1024
+DIRECTIONS = (0, 1, 2, 3)
+ESIZE = {"f16": 2, "bf16": 2, "f32": 4}
+
+
+def workload_bytes(shape, dtype: str) -> int:
+    """Algorithmic HBM bytes of one call: q,k,v read, log_alpha read (fp32),
+    out written, final state written (fp32)."""
+    tok = shape.B * shape.H * shape.tokens
+    e = ESIZE[dtype]
+    return (tok * (2 * shape.d_k + shape.d_v) * e + tok * shape.d_k * 4 + tok * shape.d_v * e
+            + shape.B * shape.H * shape.d_k * shape.d_v * 4)
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int, period_ms: int = 50):
+        self.gpu = gpu_index
+        self.period = period_ms
+        self.samples = []
+        self.proc = None
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", f"-lms={self.period}"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), line.strip()))
+
+    def stop(self, t0: float, t1: float):
+        if self.proc is None:
+            return None
+        time.sleep(self.period / 1000.0 * 2)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for ts, line in self.samples:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                rows.append((ts, float(parts[0]), float(parts[1]), parts[3:]))
+            except ValueError:
+                continue
+        window = [r for r in rows if t0 <= r[0] <= t1]
+        scope = "timed"
+        if not window:
+            window, scope = rows, "warmup+timed"
+        if not window:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in window:
+            for name, flag in zip(names, r[3][1:]):
+                if flag.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r[1] for r in window),
+                "sm_max_mhz": max(r[2] for r in window), "reasons": sorted(reasons),
+                "samples": len(window), "window": scope}
+
+
+def cpu_oracle_rate(shape, dtype, seconds: float = 10.0, max_reps: int = 20):
+    """The fp64 oracle, as it stands, on this host: tokens/s over the four
+    directions of one batch, repeated until ~`seconds` of CPU work."""
+    import oracle
+
+    q, k, v, la = make_inputs(shape, dtype, seed=0)
+    q, k, v, la = (t.double().numpy() for t in (q, k, v, la))
+    cores = oracle.max_threads()
+    reps = 0
+    t0 = time.perf_counter()
+    while True:
+        for d in DIRECTIONS:
+            oracle.forward(q, k, v, la, d, n_threads=cores)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds or reps >= max_reps:
+            break
+    tokens = reps * len(DIRECTIONS) * shape.B * shape.H * shape.tokens
+    return tokens / el, cores, reps, el
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    shape, dtype = CONFIGS[args.config]
+    rate, cores, reps, el = cpu_oracle_rate(shape, dtype, seconds=min(20.0, 2.0 + args.steps))
+    per_step_ms = 1000.0 * el / reps
+    line = {
+        "impl": "reference", "metric": METRIC, "value": rate, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": reps, "warmup": 0, "ms_per_step": per_step_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": args.config, "B": shape.B, "H": shape.H,
+                                        "grid": [shape.grid_h, shape.grid_w],
+                                        "d_k": shape.d_k, "d_v": shape.d_v,
+                                        "io_dtype": dtype, "directions": 4},
+        "cpu_baseline": {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{reps} steps x 4 directions of the full workload, {el:.1f} s"},
+        "e2e": {"value": rate, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default="640_b1", choices=sorted(CONFIGS))
+    ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    if args.impl == "reference":
+        run_reference(args)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from recurrent_vision_backbone_chunkwise_b200 import gla
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=180), device_id=dev)
+
+    shape, dtype = CONFIGS[args.config]
+    q0, k0, v0, la0 = make_inputs(shape, dtype, seed=rank)
+    call_bytes = workload_bytes(shape, dtype)
+    in_bytes = sum(t.numel() * t.element_size() for t in (q0, k0, v0, la0))
+    out_bytes = shape.B * shape.H * shape.tokens * shape.d_v * ESIZE[dtype]
+    set_bytes = in_bytes + len(DIRECTIONS) * out_bytes
+    R = max(2, math.ceil(2 * L2_BYTES / set_bytes))
+    sets = []
+    for _ in range(R):
+        ins = [t.to(dev) for t in (q0, k0, v0, la0)]
+        outs = [torch.empty((shape.B, shape.H, shape.grid_h, shape.grid_w, shape.d_v),
+                            dtype=q0.dtype, device=dev) for _ in DIRECTIONS]
+        fss = [torch.empty((shape.B, shape.H, shape.d_k, shape.d_v), dtype=torch.float32,
+                           device=dev) for _ in DIRECTIONS]
+        sets.append((ins, outs, fss))
+    chunk = 64
+    ws = torch.zeros(max(1, gla.gtr_gla_workspace_size(shape.B, shape.H, shape.grid_h,
+                                                         shape.grid_w, shape.d_k, shape.d_v,
+                                                         gla._DTYPE_CODE[q0.dtype], chunk)),
+                     dtype=torch.uint8, device=dev)
+
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(i, ev=None):
+        (q, k, v, la), outs, fss = sets[i % R]
+        for j, d in enumerate(DIRECTIONS):
+            if ev is not None:
+                ev[2 * j].record(stream)
+            gla.gtr_gla_fwd_ex(q, k, v, la, d, chunk=chunk, workspace=ws, out=outs[j],
+                               final_state=fss[j], stream=stream)
+            if ev is not None:
+                ev[2 * j + 1].record(stream)
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            step(i)
+    stream.synchronize()
+    assert gla.gtr_gla_status(stream) == 0
+
+    use_graph = not args.no_graph
+    K = args.steps
+    call_events = [[torch.cuda.Event(enable_timing=True, external=use_graph) for _ in range(8)]
+                   for _ in range(K)]
+    graph = None
+    launches0 = gla.gtr_gla_launch_count()
+    if use_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for i in range(K):
+                step(i, call_events[i])
+        launches_per_replay = gla.gtr_gla_launch_count() - launches0
+
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[0]) \
+        if os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")[0].isdigit() else local
+    sampler = ClockSampler(gpu_index)
+    sampler.start()
+    time.sleep(0.2)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    launches_before = gla.gtr_gla_launch_count()
+    start.record(stream)
+    if use_graph:
+        graph.replay()
+    else:
+        with torch.cuda.stream(stream):
+            for i in range(K):
+                step(i, call_events[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    if world > 1:
+        dist.barrier()
+    gpu_launches = (launches_per_replay if use_graph
+                    else gla.gtr_gla_launch_count() - launches_before)
+    clocks = sampler.stop(t_wall0, t_wall1)
+    assert gla.gtr_gla_status(stream) == 0
+
+    elapsed_ms = start.elapsed_time(end)
+    call_ms = [call_events[i][2 * j].elapsed_time(call_events[i][2 * j + 1])
+               for i in range(K) for j in range(len(DIRECTIONS))]
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    if graph is not None:
+        del graph
+
+    # end-to-end through the public API with pinned host buffers
+    K_e2e = min(K, 200)
+    host_in = [t.pin_memory() for t in (q0, k0, v0, la0)]
+    host_out = [torch.empty(sets[0][1][0].shape, dtype=q0.dtype).pin_memory()
+                for _ in DIRECTIONS]
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            step(i)
+        stream.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0.record(stream)
+        for i in range(K_e2e):
+            (q, k, v, la), outs, fss = sets[i % R]
+            for dst, src in zip((q, k, v, la), host_in):
+                dst.copy_(src, non_blocking=True)
+            for j, d in enumerate(DIRECTIONS):
+                gla.gtr_gla_fwd(q, k, v, la, d, out=outs[j], final_state=fss[j], stream=stream)
+                host_out[j].copy_(outs[j], non_blocking=True)
+        e1.record(stream)
+    stream.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    tokens_per_step = len(DIRECTIONS) * shape.B * shape.H * shape.tokens
+    value = world * K * tokens_per_step / (elapsed_ms / 1000.0)
+    e2e_value = world * K_e2e * tokens_per_step / (e2e_ms / 1000.0)
+    mean_call_s = statistics.mean(call_ms) / 1000.0
+    peak, peak_kind = measured_peaks()
+    achieved = call_bytes / mean_call_s / 1e9
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": elapsed_ms / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": dtype, "data": "synthetic",
+        "config": {"workload": args.config, "B": shape.B, "H": shape.H,
+                   "grid": [shape.grid_h, shape.grid_w], "tokens": shape.tokens,
+                   "d_k": shape.d_k, "d_v": shape.d_v, "chunk": chunk, "directions": 4,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": f"inputs rotate over {R} buffer sets "
+                         f"({R * set_bytes / 2**20:.0f} MiB > 126 MiB L2)",
+                   "cuda_graph": use_graph},
+        "kernel_us_per_call": {"mean": 1e6 * mean_call_s,
+                               "median": 1e3 * statistics.median(call_ms),
+                               "min": 1e3 * min(call_ms)},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "peak_source": f"{peak_kind} copy bandwidth",
+                     "bytes_per_call": call_bytes,
+                     "timed_unit": "one library call (all kernels of one direction)"},
+        "gpu_launches": int(gpu_launches),
+        "e2e": {"value": e2e_value, "unit": "tokens/s",
+                "h2d_bytes_per_step": in_bytes,
+                "d2h_bytes_per_step": len(DIRECTIONS) * out_bytes, "steps": K_e2e},
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, cores, reps, el = cpu_oracle_rate(shape, dtype, seconds=10.0)
+        line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": cores,
+                                "kind": "oracle",
+                                "sample": f"{reps} steps x 4 directions of the full "
+                                          f"workload in {el:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

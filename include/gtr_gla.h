@@ -1,0 +1,138 @@
+/*
+ * gtr_gla.h -- C ABI of the B200 (sm_100a) chunkwise key-gated linear
+ * attention forward pass, the token mixer of GTR.
+ *
+ * Operation ("GTR: Gated Token Recurrence for Efficient Dense Prediction",
+ * x-techcon article, section 架构 "architecture"): for every batch b and head
+ * h, a state S (d_k x d_v) is carried along a scan of the grid_h x grid_w
+ * patch-token grid.  At each token the gate keeps a per-key-dimension
+ * fraction alpha = exp(log_alpha) of the state (key-only gating, value-side
+ * decay fixed at 1), the token's key/value outer product is added, and the
+ * token's query reads the updated state:
+ *     S_t = diag(alpha_t) S_{t-1} + k_t^T v_t,   o_t = q_t S_t,   S_{-1} = 0.
+ * The scan direction is chosen per call; every direction reads and writes the
+ * row-major grid in place and the output is stored at each token's own grid
+ * position (the grid order is restored after the scan, same section).
+ * The sequence is evaluated chunkwise (same article, section 算子
+ * "operator"): chunks compute their own state contribution in parallel, the
+ * chunk-boundary states are passed along, and each chunk's output is then
+ * produced in parallel; the attention scores never reach global memory.
+ *
+ * Tensor layout (all device pointers, contiguous, row-major):
+ *   q, k        [B, H, grid_h, grid_w, d_k]   I/O dtype
+ *   v, out      [B, H, grid_h, grid_w, d_v]   I/O dtype
+ *   log_alpha   [B, H, grid_h, grid_w, d_k]   fp32, every value finite and <= 0
+ *   final_state [B, H, d_k, d_v]              fp32, row i = key dimension i
+ * The library never frees, retains or reallocates caller buffers.  Every
+ * base pointer must be 16-byte aligned; out must not overlap any input.
+ * No scale is applied inside (pre-scale k by 1/sqrt(d_k) if wanted).
+ * log_alpha values outside (-inf, 0] are not checked and give undefined
+ * results.
+ *
+ * Calls are asynchronous and stream-ordered; none synchronises the host
+ * except gtr_gla_status() and the allocation done by gtr_gla_fwd() when its
+ * internal workspace has to grow (do that first call outside any stream
+ * capture).
+ */
+#ifndef GTR_GLA_H
+#define GTR_GLA_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#ifndef __CUDA_RUNTIME_API_H__
+typedef struct CUstream_st *cudaStream_t;
+#endif
+
+/* ---- enums ---------------------------------------------------------- */
+
+/* Scan directions, in the pages' layer-cycle order (section 架构). */
+enum {
+    GTR_GLA_L2R = 0, /* raster order                                  */
+    GTR_GLA_R2L = 1, /* raster order reversed (whole sequence)       */
+    GTR_GLA_T2B = 2, /* column-major: columns left->right, top->bottom */
+    GTR_GLA_B2T = 3  /* column-major order reversed                  */
+};
+
+/* I/O dtypes of q, k, v and out. */
+enum { GTR_GLA_F16 = 0, GTR_GLA_BF16 = 1, GTR_GLA_F32 = 2 };
+
+/* Return codes.  Argument errors are reported before anything is launched. */
+enum {
+    GTR_GLA_OK = 0,
+    GTR_GLA_ERR_NULL = -1,        /* a required pointer is NULL                   */
+    GTR_GLA_ERR_SHAPE = -2,       /* B, H, grid_h or grid_w <= 0, or too large    */
+    GTR_GLA_ERR_HEAD_DIM = -3,    /* (d_k, d_v) not supported                     */
+    GTR_GLA_ERR_DIRECTION = -4,   /* direction not in [0, 3]                      */
+    GTR_GLA_ERR_ALIGN = -5,       /* a pointer is not 16-byte aligned             */
+    GTR_GLA_ERR_DTYPE = -6,       /* dtype not one of GTR_GLA_F16/BF16/F32        */
+    GTR_GLA_ERR_CHUNK = -7,       /* chunk length not supported for this dtype    */
+    GTR_GLA_ERR_WORKSPACE = -8,   /* workspace NULL or smaller than required      */
+    GTR_GLA_ERR_CUDA = -9,        /* a CUDA runtime call or launch failed         */
+    GTR_GLA_ERR_TIMEOUT = -10,    /* a device-side wait gave up (gtr_gla_status)  */
+    GTR_GLA_ERR_ALIAS = -11       /* out overlaps an input                        */
+};
+
+/* ---- entry points --------------------------------------------------- */
+
+/*
+ * gtr_gla_fwd -- forward pass with fp16 q/k/v/out, chunk length 64 and a
+ * workspace owned by the library (one per device, grown on demand, freed by
+ * gtr_gla_release).  Calls that share the library workspace must not run
+ * concurrently on the GPU (use one stream per device, or gtr_gla_fwd_ex with
+ * separate workspaces).
+ *   final_state may be NULL (not written).
+ *   Supported (d_k, d_v): (64, 64), (128, 128), (64, 128), (128, 64).
+ * Returns GTR_GLA_OK or a negative code; nothing is launched on error.
+ */
+int gtr_gla_fwd(const void *q, const void *k, const void *v, const float *log_alpha,
+                void *out, float *final_state, int B, int H, int grid_h, int grid_w,
+                int d_k, int d_v, int direction, cudaStream_t stream);
+
+/*
+ * gtr_gla_fwd_ex -- as gtr_gla_fwd with the I/O dtype, the chunk length and
+ * the workspace chosen by the caller.
+ *   dtype:     GTR_GLA_F16, GTR_GLA_BF16 or GTR_GLA_F32.
+ *   chunk:     tokens per chunk; 32, 64 or 128 for F16/BF16, 32 or 64 for
+ *              F32.  The result does not depend on it beyond rounding.
+ *   workspace: device buffer of at least gtr_gla_workspace_size(...) bytes,
+ *              256-byte aligned, zero-filled before its first use.  Every call
+ *              leaves it ready for the next one.  Calls that share a workspace
+ *              must not overlap on the GPU.  May be NULL only when the
+ *              required size is 0.
+ */
+int gtr_gla_fwd_ex(const void *q, const void *k, const void *v, const float *log_alpha,
+                   void *out, float *final_state, int B, int H, int grid_h, int grid_w,
+                   int d_k, int d_v, int direction, int dtype, int chunk,
+                   void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Workspace bytes gtr_gla_fwd_ex needs for this problem (0 if none). */
+size_t gtr_gla_workspace_size(int B, int H, int grid_h, int grid_w, int d_k, int d_v,
+                              int dtype, int chunk);
+
+/*
+ * gtr_gla_status -- synchronise `stream` and report the first device-side
+ * error latched by an earlier call on this device (GTR_GLA_ERR_TIMEOUT when a
+ * bounded wait inside a kernel gave up), or GTR_GLA_ERR_CUDA if the stream
+ * itself reports an error.  Clears the latched error.  Returns GTR_GLA_OK if
+ * all is well.
+ */
+int gtr_gla_status(cudaStream_t stream);
+
+/* Static, human-readable text for a return code. */
+const char *gtr_gla_strerror(int code);
+
+/* Free the library-owned workspaces (all devices).  Synchronises each one. */
+void gtr_gla_release(void);
+
+/* Number of kernels this library has launched in this process so far. */
+unsigned long long gtr_gla_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GTR_GLA_H */

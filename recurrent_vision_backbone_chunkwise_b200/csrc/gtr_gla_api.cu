@@ -1,0 +1,248 @@
+// gtr_gla_api.cu -- the C ABI of libgtr_gla.so: argument validation,
+// workspace management and dispatch to the kernels.  See include/gtr_gla.h for
+// the contract of every entry point.
+#include <atomic>
+#include <map>
+#include <mutex>
+
+#include "gla_common.cuh"
+#include "gla_internal.h"
+
+namespace gtr {
+
+static std::atomic<unsigned long long> g_launches{0};
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+int ensure_smem(const void *func, size_t bytes) {
+    static std::mutex mu;
+    static std::map<std::pair<const void *, int>, size_t> done;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return GTR_GLA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(mu);
+    auto key = std::make_pair(func, dev);
+    auto it = done.find(key);
+    if (it != done.end() && it->second >= bytes) return GTR_GLA_OK;
+    if (cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
+        cudaSuccess)
+        return GTR_GLA_ERR_CUDA;
+    done[key] = bytes;
+    return GTR_GLA_OK;
+}
+
+// Device-side error word (one per device): kernels latch the first error here.
+__device__ int g_dev_err;
+
+constexpr int kMaxDevices = 64;
+static std::mutex g_mu;
+static int *g_err_ptr[kMaxDevices];
+static void *g_ws[kMaxDevices];
+static size_t g_ws_bytes[kMaxDevices];
+
+static int current_device(int *dev) {
+    if (cudaGetDevice(dev) != cudaSuccess || *dev < 0 || *dev >= kMaxDevices)
+        return GTR_GLA_ERR_CUDA;
+    return GTR_GLA_OK;
+}
+
+// Address of this device's error word (looked up once per device).
+static int device_err_ptr(int dev, int **out) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_err_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_dev_err) != cudaSuccess) return GTR_GLA_ERR_CUDA;
+        g_err_ptr[dev] = (int *)p;
+    }
+    *out = g_err_ptr[dev];
+    return GTR_GLA_OK;
+}
+
+static size_t elem_size(int dtype) { return dtype == GTR_GLA_F32 ? 4 : 2; }
+
+static bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
+    const char *pa = (const char *)a, *pb = (const char *)b;
+    return pa < pb + nb && pb < pa + na;
+}
+
+static bool misaligned(const void *p) { return ((uintptr_t)p & 15u) != 0; }
+
+static bool head_dims_ok(int dk, int dv) {
+    return (dk == 64 || dk == 128) && (dv == 64 || dv == 128);
+}
+
+static bool chunk_ok(int dtype, int chunk) {
+    if (dtype == GTR_GLA_F32) return chunk == 32 || chunk == 64;
+    return chunk == 32 || chunk == 64;
+}
+
+static int validate_shape(int B, int H, int gh, int gw, int dk, int dv, int dtype, int chunk) {
+    if (B <= 0 || H <= 0 || gh <= 0 || gw <= 0) return GTR_GLA_ERR_SHAPE;
+    if ((long long)B * H > 65535 || (long long)gh * gw > (1LL << 22)) return GTR_GLA_ERR_SHAPE;
+    if (dtype != GTR_GLA_F16 && dtype != GTR_GLA_BF16 && dtype != GTR_GLA_F32)
+        return GTR_GLA_ERR_DTYPE;
+    if (!head_dims_ok(dk, dv)) return GTR_GLA_ERR_HEAD_DIM;
+    if (!chunk_ok(dtype, chunk)) return GTR_GLA_ERR_CHUNK;
+    return GTR_GLA_OK;
+}
+
+static int validate(const Problem &p) {
+    if (!p.q || !p.k || !p.v || !p.la || !p.out) return GTR_GLA_ERR_NULL;
+    int rc = validate_shape(p.B, p.H, p.gh, p.gw, p.dk, p.dv, p.dtype, p.chunk);
+    if (rc) return rc;
+    if (p.dir < 0 || p.dir > 3) return GTR_GLA_ERR_DIRECTION;
+    if (misaligned(p.q) || misaligned(p.k) || misaligned(p.v) || misaligned(p.la) ||
+        misaligned(p.out) || (p.final_state && misaligned(p.final_state)))
+        return GTR_GLA_ERR_ALIGN;
+    const size_t es = elem_size(p.dtype);
+    const size_t tok = (size_t)p.B * p.H * p.n;
+    const size_t nq = tok * p.dk * es, nv = tok * p.dv * es, nla = tok * p.dk * 4;
+    const size_t nfs = (size_t)p.B * p.H * p.dk * p.dv * 4;
+    if (overlaps(p.out, nv, p.q, nq) || overlaps(p.out, nv, p.k, nq) ||
+        overlaps(p.out, nv, p.v, nv) || overlaps(p.out, nv, p.la, nla))
+        return GTR_GLA_ERR_ALIAS;
+    if (p.final_state &&
+        (overlaps(p.final_state, nfs, p.out, nv) || overlaps(p.final_state, nfs, p.q, nq) ||
+         overlaps(p.final_state, nfs, p.k, nq) || overlaps(p.final_state, nfs, p.v, nv) ||
+         overlaps(p.final_state, nfs, p.la, nla)))
+        return GTR_GLA_ERR_ALIAS;
+    return GTR_GLA_OK;
+}
+
+static size_t workspace_bytes(const Problem &p) { return generic_workspace_bytes(p); }
+
+static int dispatch(const Problem &p, void *ws, cudaStream_t st) {
+    return launch_generic(p, ws, st);
+}
+
+static Problem make_problem(const void *q, const void *k, const void *v, const float *la,
+                            void *out, float *fs, int B, int H, int gh, int gw, int dk,
+                            int dv, int dir, int dtype, int chunk) {
+    Problem p;
+    p.q = q; p.k = k; p.v = v; p.la = la; p.out = out; p.final_state = fs;
+    p.B = B; p.H = H; p.gh = gh; p.gw = gw;
+    p.n = (gh > 0 && gw > 0 && (long long)gh * gw <= (1LL << 22)) ? gh * gw : 0;
+    p.dk = dk; p.dv = dv; p.dir = dir; p.dtype = dtype; p.chunk = chunk;
+    p.err = nullptr;
+    return p;
+}
+
+}  // namespace gtr
+
+using namespace gtr;
+
+extern "C" {
+
+int gtr_gla_fwd_ex(const void *q, const void *k, const void *v, const float *log_alpha,
+                   void *out, float *final_state, int B, int H, int grid_h, int grid_w,
+                   int d_k, int d_v, int direction, int dtype, int chunk, void *workspace,
+                   size_t workspace_bytes_, cudaStream_t stream) {
+    Problem p = make_problem(q, k, v, log_alpha, out, final_state, B, H, grid_h, grid_w,
+                             d_k, d_v, direction, dtype, chunk);
+    int rc = validate(p);
+    if (rc) return rc;
+    const size_t need = workspace_bytes(p);
+    if (need > 0 && (!workspace || workspace_bytes_ < need || ((uintptr_t)workspace & 255u)))
+        return GTR_GLA_ERR_WORKSPACE;
+    int dev;
+    if ((rc = current_device(&dev))) return rc;
+    if ((rc = device_err_ptr(dev, &p.err))) return rc;
+    return dispatch(p, workspace, stream);
+}
+
+int gtr_gla_fwd(const void *q, const void *k, const void *v, const float *log_alpha,
+                void *out, float *final_state, int B, int H, int grid_h, int grid_w, int d_k,
+                int d_v, int direction, cudaStream_t stream) {
+    Problem p = make_problem(q, k, v, log_alpha, out, final_state, B, H, grid_h, grid_w,
+                             d_k, d_v, direction, GTR_GLA_F16, 64);
+    int rc = validate(p);
+    if (rc) return rc;
+    int dev;
+    if ((rc = current_device(&dev))) return rc;
+    if ((rc = device_err_ptr(dev, &p.err))) return rc;
+    const size_t need = workspace_bytes(p);
+    void *ws = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        if (need > g_ws_bytes[dev]) {
+            // Growing: wait for work that may still use the old buffer, then
+            // replace it.  The new buffer starts zero-filled.
+            if (g_ws[dev]) {
+                if (cudaDeviceSynchronize() != cudaSuccess) return GTR_GLA_ERR_CUDA;
+                cudaFree(g_ws[dev]);
+                g_ws[dev] = nullptr;
+                g_ws_bytes[dev] = 0;
+            }
+            void *nw = nullptr;
+            if (cudaMalloc(&nw, need) != cudaSuccess) return GTR_GLA_ERR_CUDA;
+            if (cudaMemset(nw, 0, need) != cudaSuccess) {
+                cudaFree(nw);
+                return GTR_GLA_ERR_CUDA;
+            }
+            g_ws[dev] = nw;
+            g_ws_bytes[dev] = need;
+        }
+        ws = g_ws[dev];
+    }
+    return dispatch(p, ws, stream);
+}
+
+size_t gtr_gla_workspace_size(int B, int H, int grid_h, int grid_w, int d_k, int d_v,
+                              int dtype, int chunk) {
+    if (validate_shape(B, H, grid_h, grid_w, d_k, d_v, dtype, chunk)) return 0;
+    Problem p = make_problem(nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, B, H,
+                             grid_h, grid_w, d_k, d_v, 0, dtype, chunk);
+    return workspace_bytes(p);
+}
+
+int gtr_gla_status(cudaStream_t stream) {
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return GTR_GLA_ERR_CUDA;
+    int dev;
+    if (current_device(&dev)) return GTR_GLA_ERR_CUDA;
+    int *ep;
+    if (device_err_ptr(dev, &ep)) return GTR_GLA_ERR_CUDA;
+    int host_err = 0;
+    const int zero = 0;
+    if (cudaMemcpyFromSymbol(&host_err, g_dev_err, sizeof(int)) != cudaSuccess)
+        return GTR_GLA_ERR_CUDA;
+    if (host_err != 0 && cudaMemcpyToSymbol(g_dev_err, &zero, sizeof(int)) != cudaSuccess)
+        return GTR_GLA_ERR_CUDA;
+    if (host_err == kDevErrTimeout) return GTR_GLA_ERR_TIMEOUT;
+    return host_err ? GTR_GLA_ERR_CUDA : GTR_GLA_OK;
+}
+
+const char *gtr_gla_strerror(int code) {
+    switch (code) {
+        case GTR_GLA_OK: return "ok";
+        case GTR_GLA_ERR_NULL: return "a required pointer is NULL";
+        case GTR_GLA_ERR_SHAPE: return "B, H, grid_h or grid_w out of range";
+        case GTR_GLA_ERR_HEAD_DIM: return "unsupported (d_k, d_v)";
+        case GTR_GLA_ERR_DIRECTION: return "direction must be 0..3";
+        case GTR_GLA_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+        case GTR_GLA_ERR_DTYPE: return "unsupported dtype";
+        case GTR_GLA_ERR_CHUNK: return "unsupported chunk length";
+        case GTR_GLA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+        case GTR_GLA_ERR_CUDA: return "CUDA runtime error";
+        case GTR_GLA_ERR_TIMEOUT: return "a device-side wait timed out";
+        case GTR_GLA_ERR_ALIAS: return "output overlaps an input";
+        default: return "unknown error code";
+    }
+}
+
+void gtr_gla_release(void) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    int cur = -1;
+    cudaGetDevice(&cur);
+    for (int d = 0; d < kMaxDevices; ++d) {
+        if (!g_ws[d]) continue;
+        if (cudaSetDevice(d) == cudaSuccess) {
+            cudaDeviceSynchronize();
+            cudaFree(g_ws[d]);
+        }
+        g_ws[d] = nullptr;
+        g_ws_bytes[d] = 0;
+    }
+    if (cur >= 0) cudaSetDevice(cur);
+}
+
+unsigned long long gtr_gla_launch_count(void) { return g_launches.load(); }
+
+}  // extern "C"

@@ -1,0 +1,137 @@
+"""ctypes binding of libgtr_gla.so (argument marshalling only).
+
+Every function here has the name of the C entry point it forwards to (see
+``include/gtr_gla.h``); the arithmetic runs in the library's CUDA kernels.
+If the library is missing or cannot be loaded, importing this module raises:
+there is no CPU fallback.
+
+Tensors are torch CUDA tensors, contiguous, laid out [B, H, grid_h, grid_w, d]
+(q, k, log_alpha with d = d_k; v, out with d = d_v); the final state is
+[B, H, d_k, d_v] fp32.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgtr_gla.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with "
+        "`python -m recurrent_vision_backbone_chunkwise_b200.build` (needs nvcc)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+_vp, _int, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+_lib.gtr_gla_fwd.argtypes = [_vp] * 6 + [_int] * 7 + [_vp]
+_lib.gtr_gla_fwd.restype = _int
+_lib.gtr_gla_fwd_ex.argtypes = [_vp] * 6 + [_int] * 9 + [_vp, _sz, _vp]
+_lib.gtr_gla_fwd_ex.restype = _int
+_lib.gtr_gla_workspace_size.argtypes = [_int] * 8
+_lib.gtr_gla_workspace_size.restype = _sz
+_lib.gtr_gla_status.argtypes = [_vp]
+_lib.gtr_gla_status.restype = _int
+_lib.gtr_gla_strerror.argtypes = [_int]
+_lib.gtr_gla_strerror.restype = ctypes.c_char_p
+_lib.gtr_gla_release.argtypes = []
+_lib.gtr_gla_release.restype = None
+_lib.gtr_gla_launch_count.argtypes = []
+_lib.gtr_gla_launch_count.restype = ctypes.c_ulonglong
+
+# enums of include/gtr_gla.h
+L2R, R2L, T2B, B2T = 0, 1, 2, 3
+F16, BF16, F32 = 0, 1, 2
+_DTYPE_CODE = {torch.float16: F16, torch.bfloat16: BF16, torch.float32: F32}
+
+
+class GlaError(RuntimeError):
+    def __init__(self, code: int):
+        self.code = code
+        super().__init__(f"gtr_gla error {code}: {gtr_gla_strerror(code)}")
+
+
+def gtr_gla_strerror(code: int) -> str:
+    return _lib.gtr_gla_strerror(int(code)).decode()
+
+
+def gtr_gla_launch_count() -> int:
+    return int(_lib.gtr_gla_launch_count())
+
+
+def gtr_gla_release() -> None:
+    _lib.gtr_gla_release()
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+def gtr_gla_status(stream=None) -> int:
+    return int(_lib.gtr_gla_status(_vp(_stream_handle(stream))))
+
+
+def gtr_gla_workspace_size(B, H, grid_h, grid_w, d_k, d_v, dtype=F16, chunk=64) -> int:
+    return int(_lib.gtr_gla_workspace_size(B, H, grid_h, grid_w, d_k, d_v, dtype, chunk))
+
+
+def _ptr(t):
+    return None if t is None else _vp(t.data_ptr())
+
+
+def _shape(q, v):
+    if q.dim() != 5 or v.dim() != 5:
+        raise ValueError("q and v must be 5-D [B,H,grid_h,grid_w,d]")
+    B, H, gh, gw, dk = q.shape
+    return B, H, gh, gw, dk, v.shape[-1]
+
+
+def _alloc_out(q, v, out, final_state, want_state):
+    B, H, gh, gw, dk, dv = _shape(q, v)
+    if out is None:
+        out = torch.empty((B, H, gh, gw, dv), dtype=v.dtype, device=v.device)
+    if final_state is None and want_state:
+        final_state = torch.empty((B, H, dk, dv), dtype=torch.float32, device=v.device)
+    return out, final_state
+
+
+def gtr_gla_fwd(q, k, v, log_alpha, direction, out=None, final_state=None,
+                want_state=True, stream=None):
+    """fp16 forward, chunk 64, library-owned workspace.  Returns (out, final_state)."""
+    if q.dtype != torch.float16 or k.dtype != torch.float16 or v.dtype != torch.float16:
+        raise ValueError("gtr_gla_fwd takes fp16 q, k, v (use gtr_gla_fwd_ex for others)")
+    out, final_state = _alloc_out(q, v, out, final_state, want_state)
+    B, H, gh, gw, dk, dv = _shape(q, v)
+    rc = _lib.gtr_gla_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(out),
+                          _ptr(final_state), B, H, gh, gw, dk, dv, int(direction),
+                          _vp(_stream_handle(stream)))
+    if rc != 0:
+        raise GlaError(rc)
+    return out, final_state
+
+
+def gtr_gla_fwd_ex(q, k, v, log_alpha, direction, chunk=64, workspace=None, out=None,
+                   final_state=None, want_state=True, stream=None):
+    """Forward with the dtype taken from q and a caller workspace (allocated here
+    as a zero-filled uint8 CUDA tensor if not given).  Returns (out, final_state)."""
+    out, final_state = _alloc_out(q, v, out, final_state, want_state)
+    B, H, gh, gw, dk, dv = _shape(q, v)
+    dtype = _DTYPE_CODE.get(q.dtype)
+    if dtype is None:
+        raise ValueError(f"unsupported dtype {q.dtype}")
+    need = gtr_gla_workspace_size(B, H, gh, gw, dk, dv, dtype, chunk)
+    if workspace is None and need > 0:
+        workspace = torch.zeros(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = _lib.gtr_gla_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(out),
+                             _ptr(final_state), B, H, gh, gw, dk, dv, int(direction),
+                             dtype, int(chunk), _ptr(workspace), ws_bytes,
+                             _vp(_stream_handle(stream)))
+    if rc != 0:
+        raise GlaError(rc)
+    return out, final_state

@@ -1,0 +1,153 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Metric: err = max|gpu - ref| / max|ref| over a whole output tensor (and,
+separately, over the final state) of one (config, direction, dtype) run.
+Bounds: 5e-3 for fp16 I/O and 1e-4 for fp32 I/O (the stated tolerances),
+1e-2 for bf16 I/O (bf16 output rounding alone is up to 2^-9 ~ 2e-3 of an
+element, and the tensor-core operands are rounded to bf16 as well).
+Inputs are the seeded synthetic ones; the oracle sees the dtype-rounded
+values upcast to fp64.
+"""
+import functools
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from recurrent_vision_backbone_chunkwise_b200.inputs import CONFIGS, Shape, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f16": 5e-3, "bf16": 1e-2, "f32": 1e-4}
+
+
+@functools.lru_cache(maxsize=None)
+def gla():
+    from recurrent_vision_backbone_chunkwise_b200 import gla as g
+
+    return g
+
+
+def rel(got, ref):
+    got = got.detach().cpu().double().numpy() if hasattr(got, "detach") else got
+    d = float(np.max(np.abs(ref)))
+    return float(np.max(np.abs(got - ref))) / (d if d > 0 else 1.0)
+
+
+@functools.lru_cache(maxsize=8)
+def case(shape: Shape, dtype: str, seed: int, gates: str):
+    return make_inputs(shape, dtype, seed, gates)
+
+
+@functools.lru_cache(maxsize=16)
+def reference(shape: Shape, dtype: str, seed: int, gates: str, direction: int):
+    q, k, v, la = case(shape, dtype, seed, gates)
+    return oracle.forward(q, k, v, la, direction)
+
+
+def run_gpu(shape, dtype, seed, gates, direction, chunk=64, api="ex"):
+    q, k, v, la = (t.cuda() for t in case(shape, dtype, seed, gates))
+    g = gla()
+    if api == "fwd":
+        out, fs = g.gtr_gla_fwd(q, k, v, la, direction)
+    else:
+        out, fs = g.gtr_gla_fwd_ex(q, k, v, la, direction, chunk=chunk)
+    assert g.gtr_gla_status() == 0
+    torch.cuda.synchronize()
+    return out, fs
+
+
+def check(shape, dtype, direction, chunk=64, seed=0, gates="normal", api="ex"):
+    out, fs = run_gpu(shape, dtype, seed, gates, direction, chunk, api)
+    ref_o, ref_fs = reference(shape, dtype, seed, gates, direction)
+    assert torch.isfinite(out).all()
+    e_o, e_s = rel(out, ref_o), rel(fs, ref_fs)
+    assert e_o <= TOL[dtype], f"out err {e_o:.3e} > {TOL[dtype]}"
+    assert e_s <= TOL[dtype], f"final_state err {e_s:.3e} > {TOL[dtype]}"
+    return e_o, e_s
+
+
+@pytest.mark.parametrize("direction", [0, 1, 2, 3])
+def test_tiny_fp32(direction):
+    shape, dtype = CONFIGS["tiny"]
+    check(shape, dtype, direction)
+
+
+@pytest.mark.parametrize("direction", [0, 1, 2, 3])
+def test_640_b1_fp16_default_entry_point(direction):
+    shape, dtype = CONFIGS["640_b1"]
+    check(shape, dtype, direction, api="fwd")
+
+
+@pytest.mark.parametrize("direction", [0, 1, 2, 3])
+@pytest.mark.parametrize("cfg", ["640_b8", "1024_b1", "1024_b4", "16k_d64", "16k_d128"])
+def test_configs_fp16(cfg, direction):
+    shape, dtype = CONFIGS[cfg]
+    check(shape, dtype, direction)
+
+
+@pytest.mark.parametrize("direction", [0, 1, 2, 3])
+def test_1024_b4_stress_gates(direction):
+    shape, dtype = CONFIGS["1024_b4"]
+    check(shape, dtype, direction, gates="stress")
+
+
+@pytest.mark.parametrize("chunk", [32, 64])
+@pytest.mark.parametrize("direction", [0, 3])
+def test_chunk_sweep_16k(chunk, direction):
+    shape, dtype = CONFIGS["16k_d64"]
+    check(shape, dtype, direction, chunk=chunk)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("direction", [1, 2])
+def test_other_dtypes_640(dtype, direction):
+    shape, _ = CONFIGS["640_b1"]
+    check(shape, dtype, direction)
+
+
+@pytest.mark.parametrize("dims", [(64, 128), (128, 64)])
+def test_rectangular_head_dims(dims):
+    shape = Shape(2, 3, 24, 40, dims[0], dims[1])
+    for direction in range(4):
+        check(shape, "f16", direction, seed=5)
+
+
+@pytest.mark.parametrize("grid", [(1, 1), (1, 77), (77, 1), (5, 13), (7, 9), (3, 200), (130, 2)])
+@pytest.mark.parametrize("dtype", ["f16", "f32"])
+def test_edge_grids(grid, dtype):
+    """Single token, single row/column, N < chunk, ragged tails in scan order."""
+    shape = Shape(2, 2, grid[0], grid[1], 64, 64)
+    for direction in range(4):
+        check(shape, dtype, direction, seed=9)
+
+
+def test_memoryless_gates_match():
+    """log_alpha = -80 everywhere: the factors e^{-b} would overflow any
+    factorised form; the path must still give o_t = (q_t.k_t) v_t."""
+    shape = Shape(1, 2, 16, 20, 64, 64)
+    q, k, v, _ = make_inputs(shape, "f16", 3)
+    la = torch.full(q.shape, -80.0)
+    g = gla()
+    out, fs = g.gtr_gla_fwd_ex(q.cuda(), k.cuda(), v.cuda(), la.cuda(), 2)
+    ref_o, ref_fs = oracle.forward(q, k, v, la, 2)
+    assert rel(out, ref_o) <= 5e-3
+    assert rel(fs, ref_fs) <= 5e-3
+
+
+def test_deterministic():
+    shape, dtype = CONFIGS["1024_b1"]
+    a, sa = run_gpu(shape, dtype, 0, "normal", 2)
+    b, sb = run_gpu(shape, dtype, 0, "normal", 2)
+    assert torch.equal(a, b) and torch.equal(sa, sb)
+
+
+def test_final_state_optional_and_out_untouched_elsewhere():
+    shape, dtype = CONFIGS["640_b1"]
+    q, k, v, la = (t.cuda() for t in case(shape, dtype, 0, "normal"))
+    g = gla()
+    out, fs = g.gtr_gla_fwd(q, k, v, la, 1, want_state=False)
+    assert fs is None
+    ref_o, _ = reference(shape, dtype, 0, "normal", 1)
+    assert rel(out, ref_o) <= TOL[dtype]
