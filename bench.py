@@ -265,14 +265,14 @@ def main():
     torch.cuda.synchronize()
     t_wall0 = time.time()
     launches_before = gla.gtr_gla_launch_count()
-    start.record(stream)
-    if use_graph:
-        graph.replay()
-    else:
-        with torch.cuda.stream(stream):
+    with torch.cuda.stream(stream):  # the graph replays on the current stream
+        start.record(stream)
+        if use_graph:
+            graph.replay()
+        else:
             for i in range(K):
                 step(i, call_events[i])
-    end.record(stream)
+        end.record(stream)
     torch.cuda.synchronize()
     t_wall1 = time.time()
     if world > 1:

@@ -252,7 +252,7 @@ gla_chunk_output_kernel(const T *__restrict__ q, const T *__restrict__ k,
 size_t generic_workspace_bytes(const Problem &p) {
     const size_t nc = (size_t)(p.n + p.chunk - 1) / p.chunk;
     const size_t bh = (size_t)p.B * p.H;
-    size_t bytes = bh * nc * (size_t)p.dk * p.dv * sizeof(float);
+    size_t bytes = kWsHeaderBytes + bh * nc * (size_t)p.dk * p.dv * sizeof(float);
     bytes = (bytes + 255) & ~(size_t)255;
     bytes += bh * nc * (size_t)p.dk * sizeof(float);
     return (bytes + 255) & ~(size_t)255;
@@ -262,9 +262,10 @@ template <typename T, int DK, int DV, int C>
 static int launch_generic_t(const Problem &p, void *ws, cudaStream_t st) {
     const int nc = (p.n + C - 1) / C;
     const int bh = p.B * p.H;
-    float *dS = (float *)ws;
+    char *data = (char *)ws + kWsHeaderBytes;  // the header belongs to the fused path
+    float *dS = (float *)data;
     size_t off = ((size_t)bh * nc * DK * DV * sizeof(float) + 255) & ~(size_t)255;
-    float *gam = (float *)((char *)ws + off);
+    float *gam = (float *)(data + off);
 
     const size_t sm1 = (size_t)(2 * C * DK + C * DV) * sizeof(float);
     auto k1 = gla_chunk_state_kernel<T, DK, DV, C>;

@@ -2,8 +2,10 @@
 // libgtr_gla.so (not part of the public ABI; see include/gtr_gla.h).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
+#include <stdint.h>
 
 #include "../../include/gtr_gla.h"
 
@@ -19,12 +21,27 @@ struct Problem {
     int *err;            // device error word of the current device
 };
 
+// Every workspace starts with a fixed header that only the fused kernel uses
+// (ticket / completion counters and segment flags).  It is zero before a call
+// and zero after it; the data areas of both paths start after it.
+constexpr size_t kWsHeaderBytes = 4096;
+constexpr int kWsMaxFlags = 960;  // flag slots available in the header
+
 // Record that one kernel was launched (feeds gtr_gla_launch_count()).
 void note_launch();
 
 // Raise a kernel's dynamic shared-memory limit on the current device, once per
 // (kernel, device): later calls (e.g. inside a stream capture) touch no CUDA API.
 int ensure_smem(const void *func, size_t bytes);
+
+// Encode a [rows][cols] row-gather TMA map (tensormap.cu); 0 on success.
+int encode_rows_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int esize,
+                    uint64_t rows, int cols, bool swizzle128);
+
+// Single-kernel tensor-core path (gla_fused.cu): fp16/bf16, d_k = d_v = 64, chunk 64.
+bool fused_supported(const Problem &p);
+size_t fused_workspace_bytes(const Problem &p);
+int launch_fused(const Problem &p, void *ws, cudaStream_t st);
 
 // Three-phase CUDA-core path (gla_generic.cu): all dtypes, chunk 32 or 64.
 size_t generic_workspace_bytes(const Problem &p);

@@ -107,10 +107,15 @@ static int validate(const Problem &p) {
     return GTR_GLA_OK;
 }
 
-static size_t workspace_bytes(const Problem &p) { return generic_workspace_bytes(p); }
+// fp16/bf16 with d_k = d_v = 64 and chunk 64 run the fused tensor-core kernel;
+// everything else (fp32 I/O, other head sizes or chunk lengths) the
+// three-phase CUDA-core path.
+static size_t workspace_bytes(const Problem &p) {
+    return fused_supported(p) ? fused_workspace_bytes(p) : generic_workspace_bytes(p);
+}
 
 static int dispatch(const Problem &p, void *ws, cudaStream_t st) {
-    return launch_generic(p, ws, st);
+    return fused_supported(p) ? launch_fused(p, ws, st) : launch_generic(p, ws, st);
 }
 
 static Problem make_problem(const void *q, const void *k, const void *v, const float *la,

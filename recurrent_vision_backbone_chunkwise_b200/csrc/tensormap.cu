@@ -1,0 +1,44 @@
+// tensormap.cu -- host-side TMA descriptor encoding (cuTensorMapEncodeTiled,
+// reached through the runtime's driver entry point so the library does not
+// link libcuda directly).
+#include <mutex>
+
+#include <cudaTypedefs.h>
+
+#include "gla_internal.h"
+
+namespace gtr {
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// A 2-D view [rows][cols] of a contiguous row-major tensor, loaded one row
+// per box (TMA row gathers / single-row tiles).  16-bit tensors use the
+// 128-byte swizzle (the tensor-core operand layout); fp32 rows are unswizzled.
+int encode_rows_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int esize,
+                    uint64_t rows, int cols, bool swizzle128) {
+    auto fn = encode_fn();
+    if (!fn) return 1;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * (cuuint64_t)esize};
+    cuuint32_t box[2] = {(cuuint32_t)cols, 1};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? 0 : 1;
+}
+
+}  // namespace gtr

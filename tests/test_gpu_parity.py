@@ -151,3 +151,65 @@ def test_final_state_optional_and_out_untouched_elsewhere():
     assert fs is None
     ref_o, _ = reference(shape, dtype, 0, "normal", 1)
     assert rel(out, ref_o) <= TOL[dtype]
+
+
+def test_workspace_shared_between_paths_and_left_clean():
+    """The CUDA-core path (chunk 32) and the fused path (chunk 64) may share one
+    workspace; the fused kernel's 4 KiB synchronisation header is zero after
+    every call."""
+    shape, dtype = CONFIGS["640_b1"]
+    q, k, v, la = (t.cuda() for t in case(shape, dtype, 0, "normal"))
+    g = gla()
+    need = max(g.gtr_gla_workspace_size(1, 6, 40, 40, 64, 64, g.F16, c) for c in (32, 64))
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    ref_o, ref_s = reference(shape, dtype, 0, "normal", 3)
+    for chunk in (32, 64, 32, 64):
+        out, fs = g.gtr_gla_fwd_ex(q, k, v, la, 3, chunk=chunk, workspace=ws)
+        assert g.gtr_gla_status() == 0
+        assert rel(out, ref_o) <= TOL[dtype] and rel(fs, ref_s) <= TOL[dtype]
+        assert int(ws[:4096].count_nonzero()) == 0
+
+
+def test_cuda_graph_replay_matches_eager():
+    shape, dtype = CONFIGS["1024_b1"]
+    q, k, v, la = (t.cuda() for t in case(shape, dtype, 0, "normal"))
+    g = gla()
+    ws = torch.zeros(g.gtr_gla_workspace_size(1, 12, 64, 64, 64, 64, g.F16, 64),
+                     dtype=torch.uint8, device="cuda")
+    outs = [torch.empty_like(v) for _ in range(4)]
+    fss = [torch.empty((1, 12, 64, 64), dtype=torch.float32, device="cuda") for _ in range(4)]
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        for d in range(4):  # warm-up outside capture
+            g.gtr_gla_fwd_ex(q, k, v, la, d, workspace=ws, out=outs[d], final_state=fss[d], stream=s)
+    s.synchronize()
+    eager = [o.clone() for o in outs]
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        for d in range(4):
+            g.gtr_gla_fwd_ex(q, k, v, la, d, workspace=ws, out=outs[d], final_state=fss[d], stream=s)
+    for _ in range(3):
+        for o in outs:
+            o.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        for d in range(4):
+            assert torch.equal(outs[d], eager[d])
+    assert g.gtr_gla_status() == 0
+
+
+@pytest.mark.parametrize("direction", [0, 2])
+def test_band_of_extreme_gates(direction):
+    """Some chunks carry gate spans far beyond fp32 range of e^{-b}; those take
+    the exact score path while the rest stay factorised."""
+    shape = Shape(1, 3, 32, 48, 64, 64)
+    q, k, v, la = make_inputs(shape, "f16", 4)
+    la = la.clone()
+    la[:, :, 10:14] = -60.0
+    la[:, 1, :, 20:22] = -3.0
+    g = gla()
+    out, fs = g.gtr_gla_fwd_ex(q.cuda(), k.cuda(), v.cuda(), la.cuda(), direction)
+    assert g.gtr_gla_status() == 0
+    ref_o, ref_s = oracle.forward(q, k, v, la, direction)
+    assert rel(out, ref_o) <= 5e-3
+    assert rel(fs, ref_s) <= 5e-3
