@@ -96,8 +96,10 @@ int gtr_gla_fwd(const void *q, const void *k, const void *v, const float *log_al
  * gtr_gla_fwd_ex -- as gtr_gla_fwd with the I/O dtype, the chunk length and
  * the workspace chosen by the caller.
  *   dtype:     GTR_GLA_F16, GTR_GLA_BF16 or GTR_GLA_F32.
- *   chunk:     tokens per chunk; 32, 64 or 128 for F16/BF16, 32 or 64 for
- *              F32.  The result does not depend on it beyond rounding.
+ *   chunk:     tokens per chunk, 32 or 64.  The result does not depend on it
+ *              beyond rounding.  F16/BF16 with d_k = d_v = 64 and chunk 64 run
+ *              the fused tensor-core kernel; every other combination runs the
+ *              three-phase CUDA-core path.
  *   workspace: device buffer of at least gtr_gla_workspace_size(...) bytes,
  *              256-byte aligned, zero-filled before its first use.  Every call
  *              leaves it ready for the next one.  Calls that share a workspace
@@ -108,6 +110,29 @@ int gtr_gla_fwd_ex(const void *q, const void *k, const void *v, const float *log
                    void *out, float *final_state, int B, int H, int grid_h, int grid_w,
                    int d_k, int d_v, int direction, int dtype, int chunk,
                    void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * gtr_gla_fwd_noalloc -- as gtr_gla_fwd, but the call allocates nothing.
+ * The paper has no counterpart: this is a library convenience for callers
+ * that cannot allocate device memory while they run (a fixed, pre-planned
+ * memory budget, or host code with no device allocator of its own).
+ *   Scratch: one 12 MiB device array inside this library, held by every GPU
+ *   that loads it until the process exits, and shared by every call on that
+ *   GPU.  Calls that overlap on the GPU race on it: order them (one stream per
+ *   device, or explicit dependencies).  The array keeps the last call's
+ *   contents; the part that must start at zero is zeroed once and left zero
+ *   by every call.
+ *   Set-up: the first call on a device (made with that device current) looks
+ *   up the array's address and zeroes that part on `stream`; make that first
+ *   call before any stream capture.
+ *   Supported: fp16 q/k/v/out, d_k = d_v = 64, chunk 64 (the fused kernel);
+ *   other head sizes return GTR_GLA_ERR_HEAD_DIM, and a problem whose scratch
+ *   would exceed 12 MiB returns GTR_GLA_ERR_WORKSPACE.  Never calls cudaMalloc,
+ *   cudaFree or any allocating routine.
+ */
+int gtr_gla_fwd_noalloc(const void *q, const void *k, const void *v, const float *log_alpha,
+                        void *out, float *final_state, int B, int H, int grid_h, int grid_w,
+                        int d_k, int d_v, int direction, cudaStream_t stream);
 
 /* Workspace bytes gtr_gla_fwd_ex needs for this problem (0 if none). */
 size_t gtr_gla_workspace_size(int B, int H, int grid_h, int grid_w, int d_k, int d_v,

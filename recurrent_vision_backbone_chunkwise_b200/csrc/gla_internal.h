@@ -43,6 +43,11 @@ bool fused_supported(const Problem &p);
 size_t fused_workspace_bytes(const Problem &p);
 int launch_fused(const Problem &p, void *ws, cudaStream_t st);
 
+// Argument checks of the public entry points, and the current device's error
+// word (gtr_gla_api.cu).
+int check_problem(const Problem &p);
+int error_word(int **out);
+
 // Three-phase CUDA-core path (gla_generic.cu): all dtypes, chunk 32 or 64.
 size_t generic_workspace_bytes(const Problem &p);
 int launch_generic(const Problem &p, void *ws, cudaStream_t st);

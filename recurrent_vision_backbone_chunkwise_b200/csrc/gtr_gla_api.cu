@@ -130,6 +130,15 @@ static Problem make_problem(const void *q, const void *k, const void *v, const f
     return p;
 }
 
+int check_problem(const Problem &p) { return validate(p); }
+
+int error_word(int **out) {
+    int dev;
+    int rc = current_device(&dev);
+    if (rc) return rc;
+    return device_err_ptr(dev, out);
+}
+
 }  // namespace gtr
 
 using namespace gtr;

@@ -31,6 +31,8 @@ _lib.gtr_gla_fwd.argtypes = [_vp] * 6 + [_int] * 7 + [_vp]
 _lib.gtr_gla_fwd.restype = _int
 _lib.gtr_gla_fwd_ex.argtypes = [_vp] * 6 + [_int] * 9 + [_vp, _sz, _vp]
 _lib.gtr_gla_fwd_ex.restype = _int
+_lib.gtr_gla_fwd_noalloc.argtypes = [_vp] * 6 + [_int] * 7 + [_vp]
+_lib.gtr_gla_fwd_noalloc.restype = _int
 _lib.gtr_gla_workspace_size.argtypes = [_int] * 8
 _lib.gtr_gla_workspace_size.restype = _sz
 _lib.gtr_gla_status.argtypes = [_vp]
@@ -132,6 +134,21 @@ def gtr_gla_fwd_ex(q, k, v, log_alpha, direction, chunk=64, workspace=None, out=
                              _ptr(final_state), B, H, gh, gw, dk, dv, int(direction),
                              dtype, int(chunk), _ptr(workspace), ws_bytes,
                              _vp(_stream_handle(stream)))
+    if rc != 0:
+        raise GlaError(rc)
+    return out, final_state
+
+
+def gtr_gla_fwd_noalloc(q, k, v, log_alpha, direction, out, final_state=None, stream=None):
+    """fp16 forward that allocates nothing: the caller passes ``out`` (and
+    optionally ``final_state``); the scratch is the library's fixed device
+    array.  Returns (out, final_state)."""
+    if q.dtype != torch.float16 or k.dtype != torch.float16 or v.dtype != torch.float16:
+        raise ValueError("gtr_gla_fwd_noalloc takes fp16 q, k, v")
+    B, H, gh, gw, dk, dv = _shape(q, v)
+    rc = _lib.gtr_gla_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(out),
+                                  _ptr(final_state), B, H, gh, gw, dk, dv, int(direction),
+                                  _vp(_stream_handle(stream)))
     if rc != 0:
         raise GlaError(rc)
     return out, final_state

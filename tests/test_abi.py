@@ -95,3 +95,12 @@ def test_argument_errors_return_before_launch(gla, kw, code):
 
 def test_fp32_chunk_limits(gla):
     assert call_ex(gla, dtype=gla.F32, chunk=128) == -7
+
+
+def test_noalloc_rejects_before_touching_memory(gla):
+    vp = ctypes.c_void_p
+    args = [vp(Q), vp(K), vp(V), vp(LA), vp(OUT), vp(FS)]
+    # d = 128 is not a problem the allocation-free entry point handles
+    assert gla._lib.gtr_gla_fwd_noalloc(*args, 1, 2, 4, 4, 128, 128, 0, vp(0)) == -3
+    assert gla._lib.gtr_gla_fwd_noalloc(*args, 1, 2, 4, 4, 64, 64, 7, vp(0)) == -4
+    assert gla._lib.gtr_gla_fwd_noalloc(vp(0), *args[1:], 1, 2, 4, 4, 64, 64, 0, vp(0)) == -1
