@@ -127,7 +127,7 @@ class ClockSampler:
                 "samples": len(window), "window": scope}
 
 
-def cpu_oracle_rate(shape, dtype, seconds: float = 10.0, max_reps: int = 20):
+def cpu_oracle_rate(shape, dtype, seconds: float = 10.0, max_reps: int = 100000):
     """The fp64 oracle, as it stands, on this host: tokens/s over the four
     directions of one batch, repeated until ~`seconds` of CPU work."""
     import oracle
