@@ -466,18 +466,32 @@ __global__ void __launch_bounds__(kThreads, 2) gla_fused_kernel(const __grid_con
             float acc[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) acc[e] = 0.f;
-#pragma unroll 4
-            for (int d = 0; d < nfold; ++d) {
-                const float *src = p.agg + ((size_t)bh * p.P + (seg - 1 - d)) * 4096 + j * 64 + c0;
-                const float *sc = sAg + d * 64 + c0;
+            // the loads of kFoldBatch aggregates are all issued before any of
+            // them is consumed, so several L2 round trips overlap
+            constexpr int kFoldBatch = 4;
+            const float *base = p.agg + (size_t)bh * p.P * 4096 + j * 64 + c0;
+            for (int d0 = 0; d0 < nfold; d0 += kFoldBatch) {
+                float4 v[kFoldBatch][4];
 #pragma unroll
-                for (int q4 = 0; q4 < 16; q4 += 4) {
-                    const float4 v4 = __ldcg(reinterpret_cast<const float4 *>(src + q4));
-                    const float4 s4 = *reinterpret_cast<const float4 *>(sc + q4);
-                    acc[q4] = fmaf(s4.x, v4.x, acc[q4]);
-                    acc[q4 + 1] = fmaf(s4.y, v4.y, acc[q4 + 1]);
-                    acc[q4 + 2] = fmaf(s4.z, v4.z, acc[q4 + 2]);
-                    acc[q4 + 3] = fmaf(s4.w, v4.w, acc[q4 + 3]);
+                for (int b = 0; b < kFoldBatch; ++b) {
+                    const int d = min(d0 + b, nfold - 1);
+                    const float *src = base + (size_t)(seg - 1 - d) * 4096;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) v[b][q] = __ldcg(reinterpret_cast<const float4 *>(src + 4 * q));
+                }
+#pragma unroll
+                for (int b = 0; b < kFoldBatch; ++b) {
+                    if (d0 + b < nfold) {
+                        const float *sc = sAg + (d0 + b) * 64 + c0;
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const float4 s4 = *reinterpret_cast<const float4 *>(sc + 4 * q);
+                            acc[4 * q] = fmaf(s4.x, v[b][q].x, acc[4 * q]);
+                            acc[4 * q + 1] = fmaf(s4.y, v[b][q].y, acc[4 * q + 1]);
+                            acc[4 * q + 2] = fmaf(s4.z, v[b][q].z, acc[4 * q + 2]);
+                            acc[4 * q + 3] = fmaf(s4.w, v[b][q].w, acc[4 * q + 3]);
+                        }
+                    }
                 }
             }
 #pragma unroll
