@@ -37,6 +37,8 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 from recurrent_vision_backbone_chunkwise_b200.inputs import CONFIGS, make_inputs  # noqa: E402
+from recurrent_vision_backbone_chunkwise_b200.replicas import (  # noqa: E402
+    aggregate_rate, max_over_ranks, rank_info, replica_seed)
 
 METRIC = "GLA fwd tokens/s and µs at 1600/4096/16384 tokens; % of roofline (HBM or TC)"
 L2_BYTES = 126 * 1024 * 1024
@@ -149,8 +151,7 @@ def cpu_oracle_rate(shape, dtype, seconds: float = 10.0, max_reps: int = 100000)
 
 
 def run_reference(args):
-    rank = int(os.environ.get("RANK", "0"))
-    if rank != 0:
+    if rank_info().rank != 0:
         return
     shape, dtype = CONFIGS[args.config]
     rate, cores, reps, el = cpu_oracle_rate(shape, dtype, seconds=min(20.0, 2.0 + args.steps))
@@ -191,9 +192,8 @@ def main():
     import torch.distributed as dist
     from recurrent_vision_backbone_chunkwise_b200 import gla
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    ri = rank_info()
+    world, rank, local = ri.world, ri.rank, ri.local_rank
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
@@ -202,7 +202,7 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=180), device_id=dev)
 
     shape, dtype = CONFIGS[args.config]
-    q0, k0, v0, la0 = make_inputs(shape, dtype, seed=rank)
+    q0, k0, v0, la0 = make_inputs(shape, dtype, seed=replica_seed(0, rank))
     call_bytes = workload_bytes(shape, dtype)
     in_bytes = sum(t.numel() * t.element_size() for t in (q0, k0, v0, la0))
     out_bytes = shape.B * shape.H * shape.tokens * shape.d_v * ESIZE[dtype]
@@ -285,10 +285,7 @@ def main():
     elapsed_ms = start.elapsed_time(end)
     call_ms = [call_events[i][2 * j].elapsed_time(call_events[i][2 * j + 1])
                for i in range(K) for j in range(len(DIRECTIONS))]
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, device=dev)
     if graph is not None:
         del graph
 
@@ -316,14 +313,11 @@ def main():
         e1.record(stream)
     stream.synchronize()
     e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, device=dev)
 
     tokens_per_step = len(DIRECTIONS) * shape.B * shape.H * shape.tokens
-    value = world * K * tokens_per_step / (elapsed_ms / 1000.0)
-    e2e_value = world * K_e2e * tokens_per_step / (e2e_ms / 1000.0)
+    value = aggregate_rate(world, K, tokens_per_step, elapsed_ms)
+    e2e_value = aggregate_rate(world, K_e2e, tokens_per_step, e2e_ms)
     mean_call_s = statistics.mean(call_ms) / 1000.0
     peak, peak_kind = measured_peaks()
     achieved = call_bytes / mean_call_s / 1e9
