@@ -1,40 +1,50 @@
 // gla_fused.cu -- single-kernel chunkwise GLA forward on sm_100a tensor cores
-// (fp16 / bf16 I/O, d_k = d_v = 64, chunk 64).
+// (fp16 / bf16 I/O, d_k = d_v = 64, chunk 64), warp-specialised.
 //
 // The chunkwise reorganisation of "GTR: Gated Token Recurrence for Efficient
 // Dense Prediction" (x-techcon article, section 算子) -- chunks compute their
 // own state contribution in parallel, boundary states are passed along, each
 // chunk's output is produced in parallel, scores stay on chip -- mapped onto
-// one launch of 256-thread CTAs, two per SM:
+// one launch of 320-thread CTAs, one per SM:
 //
-//   * each CTA owns a segment of L consecutive 64-token chunks of one (b,h)
-//     (the host picks L so that the whole grid is resident at once);
-//   * pre-pass: the segment's aggregate state contribution, transposed,
-//       A_seg^T = sum_c V_c^T (k_c . e^{G_after(c) + g_c - b_c})
-//     and its gate totals are accumulated in TMEM (chunks visited last to
-//     first, so every factor is <= 1) and published to the workspace;
-//   * boundary pass: once every earlier segment of the same (b,h) has
-//     published its aggregate, the incoming state is folded in one sweep,
-//     nearest segment first: S_in = sum_j diag(e^{G(j..seg)}) A_j.  The fold
-//     order is fixed, so results are bitwise reproducible, and no segment
-//     waits on another's boundary pass (only on its pre-pass);
-//   * main pass, chunk by chunk, with the fp32 state kept in TMEM as S^T:
-//       MMA1 (tf32, M=64,N=128,K=64):  [scores | o] = Q^ [K~ ; S_in^T]^T
-//         Q^ = q . e^{b},  K~ = k . e^{-b}   (b: in-chunk inclusive log-gate sums)
-//       causal mask of the scores on CUDA cores, re-quantised to f16/bf16,
-//       MMA2a (f16/bf16, M=64,N=64,K=64):  o += A V
-//       MMA2b (f16/bf16, M=64,N=64,K=64):  dS^T = V^T K^,  K^ = k . e^{g - b}
-//       S^T <- S^T diag(e^{g}) + dS^T;  o stored at the tokens' raster rows.
-//     The gate factors come from running products of alpha = e^{log_alpha}
-//     (one exponential per element).
-//   Chunks whose in-chunk gate span exceeds kSpanLimit (e^{-b} would leave
-//   fp32 range) take an exact CUDA-core path for the scores.
+//   * a CTA owns a segment of L consecutive 64-token chunks of one (b,h);
+//     CTAs take their segment from a ticket counter, so a segment only ever
+//     waits for segments that were started before it;
+//   * pre-pass (every segment but the last of its (b,h)): the segment's
+//     aggregate state contribution, transposed,
+//       A_seg^T = sum_c V_c^T (k_c . e^{G_after(c) + g_c - b_c}),
+//     accumulates in TMEM (chunks visited last to first, every factor <= 1)
+//     and is published with the segment's gate totals;
+//   * boundary: the incoming state is the fold of every earlier segment's
+//     aggregate, nearest first, S_in = sum_j diag(e^{G(j..seg)}) A_j (a fixed
+//     order: results are bitwise reproducible);
+//   * main pass, chunk by chunk:
+//       scores = Q^ K~^T        (tf32 MMA; Q^ = q . e^{b}, K~ = k . e^{-b},
+//                                b: in-chunk inclusive log-gate sums)
+//       dS^T   = V^T K^         (f16/bf16 MMA; K^ = k . e^{g - b})
+//       A      = causal mask of the scores, re-quantised to the I/O dtype
+//       o      = Q^ S_in + A V  (tf32 + f16/bf16 MMAs into one accumulator)
+//       S      <- diag(e^{g}) S + dS   (fp32, registers of the epilogue warps)
 //
-// Tiles are fetched in scan order by cp.async row copies (a per-chunk table of
-// raster rows), so every scan direction reads and writes the row-major grid in
-// place.  Every M=64 result lands in TMEM lanes 32(r/16) + r%16 (lanes 0-15
-// of each warp's quadrant), so row r is handled by lane r%16 of the warps of
-// quadrant r/16; each of the two warps of a quadrant takes 32 columns.
+// Roles (warps):
+//   0      producer: row tables and TMA row gathers of q, k, v, log_alpha into
+//          a 3-stage ring (rows fetched in scan order, so every direction
+//          reads and writes the row-major grid in place);
+//   1      MMA issue (one lane) and TMEM allocation;
+//   2..5   operand warps: gate factors (one exponential per element, running
+//          products), Q^ / K~ (tf32, written over log_alpha / q,k in place)
+//          and K^ (f16/bf16), 16 token rows each;
+//   6..9   epilogue warps, one per TMEM lane quadrant: causal mask, state
+//          update (state in registers, a tf32 copy in shared memory as the
+//          next chunk's MMA operand), output stores, the fold, the
+//          aggregate's publication.
+// Chunk k's scores and dS are issued as soon as its operands are ready, ahead
+// of chunk k-1's output product, so the only serial chain from chunk to chunk
+// is the epilogue's state update.
+//
+// Chunks whose in-chunk gate span exceeds kSpanLimit (e^{-b} would leave fp32
+// range) get their scores from an exact CUDA-core evaluation by the operand
+// warps (every factor <= 1), stored straight into TMEM.
 #include <type_traits>
 
 #include "gla_common.cuh"
@@ -46,47 +56,61 @@ using namespace sm100;
 
 namespace {
 
-constexpr int FC = 64;              // tokens per chunk
-constexpr int FD = 64;              // d_k = d_v
-constexpr int kThreads = 256;       // 8 warps: two per TMEM lane quadrant
-constexpr int kMaxSegments = 64;    // segments per (b,h); bounds the look-back fold
+constexpr int FC = 64;  // tokens per chunk
+constexpr int FD = 64;  // d_k = d_v
+constexpr int kStages = 3;
+constexpr int kThreads = 320;
+constexpr int kWarpLoad = 0, kWarpMma = 1, kWarpOp0 = 2, kWarpEpi0 = 6;
+constexpr int kOpThreads = 128, kEpiThreads = 128;
+constexpr int kBarOp = 1, kBarEpi = 2;  // named barrier ids
+constexpr int kMaxSegments = 64;        // segments per (b,h): bounds the fold
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kSpanLimit = 80.f;  // max -g (natural log) for the factorised scores
 
-// shared-memory map (byte offsets from a 1024-aligned base)
-constexpr uint32_t OFF_Q = 0;        // q tile    [64 tok][128 B]  SW128
-constexpr uint32_t OFF_K = 8192;     // k tile    [64 tok][128 B]  SW128
-constexpr uint32_t OFF_V = 16384;    // v tile    [64 tok][128 B]  SW128 (MMA2 B, MN-major)
-constexpr uint32_t OFF_LA = 24576;   // log_alpha [64 tok][256 B]  fp32
-constexpr uint32_t OFF_QH = 40960;   // MMA1 A:  Q^ tf32 K-major [kc 2][64][128 B]
-constexpr uint32_t OFF_B1 = 57344;   // MMA1 B: tf32 K-major [kc 2][128 rows][128 B]:
-                                     //   rows 0-63 K~ (tokens), rows 64-127 S_in^T (value dims)
-constexpr uint32_t OFF_A = 90112;    // A (masked scores) f16/bf16 K-major [64 t][128 B]
-constexpr uint32_t OFF_KH = 98304;   // K^ f16/bf16 K-major [64 i][128 B]
-constexpr uint32_t OFF_MISC = 106496;
-// pre-pass stage 1 (the operand tiles are idle during the pre-pass)
-constexpr uint32_t OFF_K1 = OFF_QH, OFF_V1 = OFF_QH + 8192, OFF_LA1 = OFF_B1;
-constexpr uint32_t MISC_TOT = 0;     // [8][64] fp32 row-group totals of log_alpha
-constexpr uint32_t MISC_G = 2048;    // [64] fp32 e^{g} of the current chunk
-constexpr uint32_t MISC_GA = 2304;   // [64] fp32 pre-pass: gate sums of later chunks
-constexpr uint32_t MISC_ROW = 2816;  // [2][64] int: global row index of each token of a chunk
+// One pipeline stage (byte offsets from the stage base, every tile 1024-aligned).
+constexpr uint32_t ST_Q = 0;       // q  [64 tok][128 B] plain rows; later K~ (tf32, 16 KB, with ST_K)
+constexpr uint32_t ST_K = 8192;    // k  [64 tok][128 B] plain rows
+constexpr uint32_t ST_V = 16384;   // v  [64 tok][128 B] SW128 (MN-major MMA operand)
+constexpr uint32_t ST_LA = 24576;  // log_alpha [64 tok][256 B] fp32; later Q^ (tf32, 16 KB)
+constexpr uint32_t ST_KH = 40960;  // K^ [64 i][128 B] SW128 K-major
+constexpr uint32_t ST_BYTES = 49152;
+constexpr uint32_t ST_KT = ST_Q, ST_QH = ST_LA;
+constexpr uint32_t OFF_SB = kStages * ST_BYTES;  // S^T tf32 K-major [2][16 KB]
+constexpr uint32_t OFF_A = OFF_SB + 2 * 16384;   // A f16/bf16 K-major [2][8 KB]
+constexpr uint32_t OFF_MISC = OFF_A + 2 * 8192;
+constexpr uint32_t MISC_ROWS = 0;     // int   [kStages][64] global row of each token
+constexpr uint32_t MISC_GAM = 768;    // float [kStages][64] e^{g}
+constexpr uint32_t MISC_TOT = 1536;   // float [2][4][64] operand warps' row-block log sums
+constexpr uint32_t MISC_LEN = 3584;   // int   [kStages] tokens in the chunk
+constexpr uint32_t MISC_FLAG = 3600;  // int   [kStages] exact-score chunk
 constexpr uint32_t MISC_BYTES = 4096;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
-constexpr uint32_t kTmemCols = 256;
-// TMEM columns (all M=64 results): scores, output o, dS^T, state S^T
-constexpr uint32_t TM_RAW = 0, TM_O = 64, TM_DS = 128, TM_S = 192;
+static_assert(SMEM_BYTES <= 232448, "shared memory");
+
+constexpr uint32_t kTmemCols = 512;
+// TMEM columns (M = 64 results, lanes 32 q + 0..15): scores, dS^T, o (two
+// buffers each, by chunk parity) and the pre-pass aggregate.
+constexpr uint32_t TM_SC = 0, TM_DS = 128, TM_O = 256, TM_PRE = 384;
 
 struct FusedParams {
+    // Tiled views of q, k, v, log_alpha.  Row scans (L->R, R->L): [BH][n][64],
+    // one 64-row box per chunk.  Column scans (T->B, B->T): [BH][gh][gw][64],
+    // boxes of `boxh` consecutive grid rows of one column (boxh: the largest
+    // power of two <= 64 that divides grid_h, so no box crosses a column).
+    CUtensorMap tm_q, tm_k, tm_v, tm_la;
     const void *q, *k, *v;
     const float *la;
     void *out;
     float *final_state;
-    float *agg;    // [BH*P][64*64] segment aggregate states, transposed ([j][i])
-    float *aggg;   // [BH*P][64]    segment log-gate totals
-    int *flag;     // [BH*P] 0 empty, 1 aggregate published
-    unsigned *ctr; // [0] ticket, [1] finished CTAs
+    float *agg;     // [BH*P][64*64] segment aggregate states, transposed ([j][i])
+    float *aggg;    // [BH*P][64]    segment log-gate totals
+    int *flag;      // [BH*P] 0 empty, 1 aggregate published
+    unsigned *ctr;  // [0] ticket, [1] finished CTAs
     int *err;
     int n, gh, gw, dir, nc, P, L, BH;
+    int boxh;  // rows per box (64 for row scans); 0: four-row gathers (column
+               // scans whose grid_h is not a multiple of 8, where a box of V
+               // could not start on its 128-byte swizzle atom)
 };
 
 __device__ __forceinline__ int ld_acquire(const int *p) {
@@ -99,18 +123,48 @@ __device__ __forceinline__ void st_release(int *p, int v) {
     asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-// Bounded wait (about 2 s) for a non-zero flag; 0 (and a latched error) if it
-// never came.
-__device__ int wait_flag(const int *f, int *err) {
+// Bounded wait (about 2 s) for a non-zero flag; false if it never came.
+__device__ bool wait_flag(const int *f) {
     const uint64_t t0 = global_timer_ns();
     while (true) {
-        const int v = ld_acquire(f);
-        if (v != 0) return v;
-        if (global_timer_ns() - t0 > 2000000000ull) break;
-        __nanosleep(32);
+        if (ld_acquire(f) != 0) return true;
+        if (global_timer_ns() - t0 > 2000000000ull) return false;
+        __nanosleep(64);
     }
-    latch_error(err, kDevErrTimeout);
-    return 0;
+}
+
+// Polling side of a pipeline wait, bounded (about 2 s): the first wait that
+// gives up raises `abort`, after which every wait returns at once, so all
+// threads reach the end of the kernel.  It spins on try_wait for about a
+// microsecond, then backs off with short sleeps (from the start when
+// `sleep_ns` is set): a waiting warp must not take issue slots from the
+// warps doing the work.  Returns false when aborted.
+__device__ bool pwait(uint64_t *bar, uint32_t parity, volatile int *abort, int *err,
+                      uint32_t sleep_ns = 0) {
+    if (mbar_test_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t n = 0;; ++n) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((n & 7) == 7) {
+            if (*abort) return false;
+            const uint64_t dt = global_timer_ns() - t0;
+            if (dt > 2000000000ull) {
+                *abort = 1;
+                latch_error(err, kDevErrTimeout);
+                return false;
+            }
+            if (sleep_ns || dt > 1000) __nanosleep(sleep_ns ? sleep_ns : 64);
+        }
+    }
+}
+
+// A group of warps waits through one polling thread; the group's named
+// barrier (id, count threads) releases the others.  Returns false when aborted.
+__device__ __forceinline__ bool gwait(bool leader, int id, int count, uint64_t *bar, uint32_t parity,
+                                      volatile int *abort, int *err, uint32_t sleep_ns = 0) {
+    if (leader) pwait(bar, parity, abort, err, sleep_ns);
+    named_bar_sync(id, count);
+    return *abort == 0;
 }
 
 template <typename T> struct Pack2;
@@ -133,25 +187,6 @@ template <> struct Pack2<__nv_bfloat16> {
     }
 };
 
-// element (row, col) of a [rows][64] 16-bit SW128 tile
-template <typename T>
-__device__ __forceinline__ float tile16(const uint8_t *tile, int row, int col) {
-    return to_f32(*reinterpret_cast<const T *>(tile + sw128(row, col >> 3) + (col & 7) * 2));
-}
-
-// byte offset of tf32 element (row, k) in a K-major tile with K = 64 and
-// `rows` rows per 32-element K block
-template <int rows>
-__device__ __forceinline__ uint32_t tf32_kmaj(int row, int k) {
-    return (k >> 5) * (rows * 128) + sw128(row, (k & 31) >> 2) + (k & 3) * 4;
-}
-
-// A shared-memory descriptor advanced by `bytes` (the start address field
-// holds addr >> 4 in its low 14 bits; smem addresses stay far below 256 KiB).
-__device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) {
-    return d + (uint64_t)(bytes >> 4);
-}
-
 template <typename T>
 __device__ __forceinline__ uint4 pack8(const float *x) {
     uint4 w;
@@ -162,134 +197,66 @@ __device__ __forceinline__ uint4 pack8(const float *x) {
     return w;
 }
 
-// One thread waits (bounded) for an mbarrier phase, then the CTA barrier
-// releases everyone: waiting warps sleep in bar.sync instead of spinning.
-// Must be reached by every thread.  Returns false if the wait gave up (or an
-// earlier one did: then nobody waits any more).
-__device__ __forceinline__ bool cta_wait(uint64_t *bar, uint32_t parity, bool ok, int *s_ok) {
-    if (threadIdx.x == 0) *s_ok = (ok && mbar_wait(bar, parity)) ? 1 : 0;
-    __syncthreads();
-    return *s_ok != 0;
+// byte offset of tf32 element (row, k) in a K-major [2 blocks of 32][64 rows][128 B] tile
+__device__ __forceinline__ uint32_t tf32_kmaj(int row, int k) {
+    return (k >> 5) * 8192 + sw128(row, (k & 31) >> 2) + (k & 3) * 4;
 }
 
-// Global row (b,h plane offset included) of every token of chunk c, in scan
-// order; rows past the end of the sequence repeat the last token (they are
-// masked in the arithmetic).  Threads 0..63 fill one table.
-__device__ __forceinline__ void fill_rows(const FusedParams &p, int bh, int c, int *rows) {
-    const int u = threadIdx.x;
-    if (u < FC)
-        rows[u] = bh * p.n + scan_to_raster(min(c * FC + u, p.n - 1), p.n, p.gh, p.gw, p.dir);
+// A shared-memory descriptor advanced by `bytes` (the start address field
+// holds addr >> 4 in its low 14 bits; smem addresses stay far below 256 KiB).
+__device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) {
+    return d + (uint64_t)(bytes >> 4);
 }
 
-// cp.async copies of a 64-row tile of 16-bit [.., 64] rows into a SW128 tile
-// (2 pieces of 16 B per thread).
-__device__ __forceinline__ void copy_tile16(uint8_t *dst, const void *src, const int *rows) {
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-        const int pc = threadIdx.x + kThreads * e;
-        const int u = pc >> 3, w = pc & 7;
-        cp_async16(dst + sw128(u, w),
-                   static_cast<const uint8_t *>(src) + (size_t)rows[u] * 128 + w * 16);
-    }
-}
-
-// cp.async copies of a 64-row tile of fp32 [.., 64] rows (4 pieces per thread).
-__device__ __forceinline__ void copy_tile32(uint8_t *dst, const float *src, const int *rows) {
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        const int pc = threadIdx.x + kThreads * e;
-        const int u = pc >> 4, w = pc & 15;
-        cp_async16(dst + u * 256 + w * 16,
-                   reinterpret_cast<const uint8_t *>(src) + (size_t)rows[u] * 256 + w * 16);
-    }
-}
-
-// Gate factors of a 64-token chunk for the columns (p2, p2+1) and the rows
-// [8 r8, 8 r8 + 8) of this thread: alpha = e^{log_alpha} per element, the
-// chunk's log-gate totals g (returned), and the row-group log sums that place
-// the thread's rows inside the chunk (pre: groups before, suf: groups after).
-// Rows >= len count as alpha = 1.  Contains one __syncthreads.
-struct GateRows {
-    float a0[8], a1[8];  // alpha of the 8 rows, columns p2 and p2+1
-    float pre0, pre1;    // sum of log_alpha over the rows before this group
-    float suf0, suf1;    // sum of log_alpha over the rows after this group
-    float g0, g1;        // chunk totals
-};
-
-__device__ __forceinline__ void gate_rows(const float *sLA, float *sTot, int p2, int r8, int len,
-                                          GateRows &G) {
-    float l0 = 0.f, l1 = 0.f;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-        const int u = 8 * r8 + k;
-        float2 x = make_float2(0.f, 0.f);
-        if (u < len) x = *reinterpret_cast<const float2 *>(sLA + u * 64 + p2);
-        l0 += x.x;
-        l1 += x.y;
-        G.a0[k] = fast_exp2(x.x * kLog2e);
-        G.a1[k] = fast_exp2(x.y * kLog2e);
-    }
-    *reinterpret_cast<float2 *>(sTot + r8 * 64 + p2) = make_float2(l0, l1);
-    __syncthreads();
-    float o0 = 0.f, o1 = 0.f, t0 = 0.f, t1 = 0.f;
-#pragma unroll
-    for (int gidx = 0; gidx < 8; ++gidx) {
-        const float2 t = *reinterpret_cast<const float2 *>(sTot + gidx * 64 + p2);
-        if (gidx < r8) {
-            o0 += t.x;
-            o1 += t.y;
-        }
-        t0 += t.x;
-        t1 += t.y;
-    }
-    G.pre0 = o0;
-    G.pre1 = o1;
-    G.suf0 = t0 - o0 - l0;
-    G.suf1 = t1 - o1 - l1;
-    G.g0 = t0;
-    G.g1 = t1;
+__device__ __forceinline__ float2 ld2(const float *p) { return *reinterpret_cast<const float2 *>(p); }
+__device__ __forceinline__ void st2(float *p, float2 v) { *reinterpret_cast<float2 *>(p) = v; }
+__device__ __forceinline__ float2 ex2_2(float2 x) {
+    return make_float2(fast_exp2(x.x * kLog2e), fast_exp2(x.y * kLog2e));
 }
 
 template <bool BF16>
-__global__ void __launch_bounds__(kThreads, 2) gla_fused_kernel(const __grid_constant__ FusedParams p) {
+__global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_constant__ FusedParams p) {
     using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    uint8_t *sQ = sm + OFF_Q, *sK = sm + OFF_K, *sV = sm + OFF_V;
-    float *sLA = reinterpret_cast<float *>(sm + OFF_LA);
-    uint8_t *sQH = sm + OFF_QH, *sB1 = sm + OFF_B1;
-    uint8_t *sA = sm + OFF_A, *sKh = sm + OFF_KH;
+    // 1024-aligned base; offset arithmetic on the array keeps shared-memory
+    // accesses in the shared state space (no generic loads)
+    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    int *sRows = reinterpret_cast<int *>(sm + OFF_MISC + MISC_ROWS);
+    float *sGam = reinterpret_cast<float *>(sm + OFF_MISC + MISC_GAM);
     float *sTot = reinterpret_cast<float *>(sm + OFF_MISC + MISC_TOT);
-    float *sGam = reinterpret_cast<float *>(sm + OFF_MISC + MISC_G);  // e^{g} of the chunk
-    float *sGa = reinterpret_cast<float *>(sm + OFF_MISC + MISC_GA);
-    int *sRow = reinterpret_cast<int *>(sm + OFF_MISC + MISC_ROW);  // [2][64]
+    int *sLen = reinterpret_cast<int *>(sm + OFF_MISC + MISC_LEN);
+    int *sFlag = reinterpret_cast<int *>(sm + OFF_MISC + MISC_FLAG);
 
-    // bar_st: pre-pass stages; bar_ld / bar_v: main-pass q,k,log_alpha / v.
-    __shared__ uint64_t bar_st[2], bar_ld, bar_v, bar_mma;
+    __shared__ uint64_t bar_full[kStages], bar_empty[kStages], bar_op[kStages];
+    __shared__ uint64_t bar_sc[2], bar_o[2], bar_a[2], bar_s[2];
+    __shared__ uint64_t bar_pre, bar_owpre, bar_fin;
     __shared__ uint32_t s_tmem;
-    __shared__ int s_ticket, s_last, s_fail, s_ok;
+    __shared__ int s_ticket, s_last;
+    __shared__ volatile int s_abort;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quad = warp & 3, ch = warp >> 2;  // TMEM lane quadrant, column half
-    const bool act = lane < 16;                 // lanes holding M=64 rows
-    const int row16 = 16 * quad + (lane & 15);  // row of the M=64 results this lane holds
-    const uint32_t lane_off = (uint32_t)(32 * quad) << 16;
-    const int p2 = 2 * (tid & 31), r8 = tid >> 5;  // gate math: columns p2, p2+1; rows 8 r8..
-    constexpr uint32_t kFmt = BF16 ? 1u : 0u;
-    const uint32_t id_tf = idesc(2, 64, 128, 0, 0);     // tf32, both K-major, N = 128
-    const uint32_t id_av = idesc(kFmt, 64, 64, 0, 1);   // A K-major, V as B (MN-major)
-    const uint32_t id_vk = idesc(kFmt, 64, 64, 1, 0);   // V^T as A (MN-major), K^ as B
 
     if (tid == 0) {
-        mbar_init(&bar_st[0], kThreads);
-        mbar_init(&bar_st[1], kThreads);
-        mbar_init(&bar_ld, kThreads);
-        mbar_init(&bar_v, kThreads);
-        mbar_init(&bar_mma, 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&bar_full[s], 1);  // producer lane 0 (with the stage's TMA bytes)
+            mbar_init(&bar_empty[s], 1);
+            mbar_init(&bar_op[s], kOpThreads);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&bar_sc[b], 1);
+            mbar_init(&bar_o[b], 1);
+            mbar_init(&bar_a[b], kEpiThreads);
+            mbar_init(&bar_s[b], kEpiThreads);
+        }
+        mbar_init(&bar_pre, 1);
+        mbar_init(&bar_owpre, kOpThreads);
+        mbar_init(&bar_fin, 1);
         fence_mbar_init();
         s_ticket = (int)atomicAdd(&p.ctr[0], 1u);
+        s_abort = 0;
     }
-    if (warp == 1) {
+    for (int e = tid; e < kStages * 64; e += kThreads) sRows[e] = 0;
+    if (warp == kWarpMma) {
         tmem_alloc(&s_tmem, kTmemCols);
         tmem_relinquish();
     }
@@ -300,473 +267,540 @@ __global__ void __launch_bounds__(kThreads, 2) gla_fused_kernel(const __grid_con
     const int ticket = s_ticket;
     const int bh = ticket / p.P, seg = ticket % p.P;
     const int c_begin = seg * p.L, c_end = min(c_begin + p.L, p.nc);
+    const int L = c_end - c_begin;
+    const int npre = (seg < p.P - 1) ? L : 0;  // the last segment needs no aggregate
+    const int n_items = npre + L;
     const size_t slot = (size_t)bh * p.P + seg;
+    constexpr uint32_t kFmt = BF16 ? 1u : 0u;
 
-    uint32_t ph_st0 = 0, ph_st1 = 0, ph_ld = 0, ph_v = 0, ph_mma = 0;
-    bool ok = true;  // every bounded wait succeeded
-
-    // ------------------------------------------------------------- pre-pass
-    // A_seg^T accumulates in TM_DS:  sum_c V_c^T (k_c . e^{G_after + g_c - b})
-    if (seg < p.P - 1) {
-        const int nl = c_end - c_begin;
-        if (tid < 64) sGa[tid] = 0.f;
-        fill_rows(p, bh, c_end - 1, sRow);
-        if (nl > 1) fill_rows(p, bh, c_end - 2, sRow + 64);
-        __syncthreads();
-        copy_tile16(sK, p.k, sRow);
-        copy_tile32(reinterpret_cast<uint8_t *>(sLA), p.la, sRow);
-        copy_tile16(sV, p.v, sRow);
-        cp_async_arrive(&bar_st[0]);
-        if (nl > 1) {
-            copy_tile16(sm + OFF_K1, p.k, sRow + 64);
-            copy_tile32(sm + OFF_LA1, p.la, sRow + 64);
-            copy_tile16(sm + OFF_V1, p.v, sRow + 64);
-            cp_async_arrive(&bar_st[1]);
+    if (warp == kWarpLoad) {
+        // ------------------------------------------------------------ producer
+        // TMA tile loads of whole chunks: one box per tensor for row scans,
+        // FC / boxh column slabs per tensor for column scans.
+        const uint64_t pol_keep = l2_policy_evict_last();  // pre-pass data is read again
+        const uint64_t pol_once = l2_policy_evict_first();
+        if (lane == 0) {
+            tma_prefetch_desc(&p.tm_q);
+            tma_prefetch_desc(&p.tm_k);
+            tma_prefetch_desc(&p.tm_v);
+            tma_prefetch_desc(&p.tm_la);
         }
-        for (int idx = 0; idx < nl; ++idx) {
-            const int c = c_end - 1 - idx, st = idx & 1;
-            const int len = min(FC, p.n - c * FC);
-            const uint8_t *kt = st ? sm + OFF_K1 : sK;
-            const float *lat = reinterpret_cast<const float *>(st ? sm + OFF_LA1 : sm + OFF_LA);
-            const uint8_t *vt = st ? sm + OFF_V1 : sV;
-            if (st == 0) {
-                ok = cta_wait(&bar_st[0], ph_st0, ok, &s_ok);
-                ph_st0 ^= 1;
-            } else {
-                ok = cta_wait(&bar_st[1], ph_st1, ok, &s_ok);
-                ph_st1 ^= 1;
+        bool ok = true;
+        uint32_t issued = 0;  // bit s: the last use of stage s had its copies issued
+        for (int it = 0; it < n_items; ++it) {
+            const int s = it % kStages;
+            const bool pre = it < npre;
+            const int c = pre ? (c_end - 1 - it) : (c_begin + it - npre);
+            if (it >= kStages) {
+                bool w = true;
+                if (lane == 0) w = pwait(&bar_empty[s], ((it / kStages) - 1) & 1, &s_abort, p.err, 64);
+                ok = __shfl_sync(0xffffffffu, w, 0) && ok;
             }
-            GateRows G;
-            gate_rows(lat, sTot, p2, r8, len, G);
-            {
-                const float2 ga = *reinterpret_cast<const float2 *>(sGa + p2);
-                // e^{G_after + g - b_u} = e^{G_after} * prod of the alphas after u
-                float e0 = fast_exp2((ga.x + G.suf0) * kLog2e), e1 = fast_exp2((ga.y + G.suf1) * kLog2e);
-                float kh0[8], kh1[8];
+            issued = ok ? (issued | (1u << s)) : (issued & ~(1u << s));
+            // row table (for the output stores): global row of every token
+            int *rows = sRows + s * 64;
 #pragma unroll
-                for (int k = 7; k >= 0; --k) {
-                    const int u = 8 * r8 + k;
-                    float2 kv = make_float2(0.f, 0.f);
-                    if (u < len)
-                        kv = Pack2<T>::unpack(*reinterpret_cast<const uint32_t *>(
-                            kt + sw128(u, p2 >> 3) + (p2 & 7) * 2));
-                    kh0[k] = kv.x * e0;
-                    kh1[k] = kv.y * e1;
-                    e0 *= G.a0[k];
-                    e1 *= G.a1[k];
+            for (int e = 0; e < 2; ++e) {
+                const int u = lane + 32 * e;
+                rows[u] = bh * p.n + scan_to_raster(min(c * FC + u, p.n - 1), p.n, p.gh, p.gw, p.dir);
+            }
+            if (lane == 0) sLen[s] = min(FC, p.n - c * FC);
+            __syncwarp();
+            if (lane == 0) mbar_arrive_expect_tx(&bar_full[s], pre ? 32768u : 40960u);
+            __syncwarp();
+            // The chunk's tokens, in stage-row order: row scans load raster rows
+            // [y0, y0+64) of the plane, column scans the column-major positions
+            // [p0, p0+64); reversed scans take the same range read backwards
+            // (token u sits in stage row 63 - u).  Rows outside the grid read
+            // as zero.
+            if (ok) {
+                uint8_t *st = sm + s * ST_BYTES;
+                const uint64_t pol = pre ? pol_keep : pol_once;
+                const int p0 = (p.dir & 1) ? (p.n - FC - c * FC) : c * FC;
+                if (p.dir < 2) {
+                    if (lane == 0) {
+                        tma_load_3d_pol(st + ST_K, &p.tm_k, &bar_full[s], 0, p0, bh, pol);
+                        tma_load_3d_pol(st + ST_V, &p.tm_v, &bar_full[s], 0, p0, bh, pol);
+                        tma_load_3d_pol(st + ST_LA, &p.tm_la, &bar_full[s], 0, p0, bh, pol);
+                        if (!pre) tma_load_3d_pol(st + ST_Q, &p.tm_q, &bar_full[s], 0, p0, bh, pol_once);
+                    }
+                } else if (p.boxh == 0) {
+                    if (lane < 16) {  // stage rows 4 lane .. 4 lane + 3, as row gathers
+                        int r[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int u = (p.dir & 1) ? 63 - (4 * lane + e) : 4 * lane + e;
+                            r[e] = bh * p.n + scan_to_raster(min(c * FC + u, p.n - 1), p.n, p.gh, p.gw, p.dir);
+                        }
+                        const int m = 4 * lane;
+                        tma_gather4_pol(st + ST_K + m * 128, &p.tm_k, &bar_full[s], 0, r[0], r[1], r[2], r[3], pol);
+                        tma_gather4_pol(st + ST_V + m * 128, &p.tm_v, &bar_full[s], 0, r[0], r[1], r[2], r[3], pol);
+                        tma_gather4_pol(st + ST_LA + m * 256, &p.tm_la, &bar_full[s], 0, r[0], r[1], r[2], r[3], pol);
+                        if (!pre)
+                            tma_gather4_pol(st + ST_Q + m * 128, &p.tm_q, &bar_full[s], 0, r[0], r[1], r[2], r[3],
+                                            pol_once);
+                    }
+                } else {
+                    const int h = p.boxh;
+                    for (int bx = lane; bx < FC / h; bx += 32) {
+                        const int pp = p0 + bx * h;  // a multiple of h: the box stays in one column
+                        const int x = pp >= 0 ? pp / p.gh : -1, y = pp >= 0 ? pp % p.gh : 0;
+                        const int r = bx * h;
+                        tma_load_4d_pol(st + ST_K + r * 128, &p.tm_k, &bar_full[s], 0, x, y, bh, pol);
+                        tma_load_4d_pol(st + ST_V + r * 128, &p.tm_v, &bar_full[s], 0, x, y, bh, pol);
+                        tma_load_4d_pol(st + ST_LA + r * 256, &p.tm_la, &bar_full[s], 0, x, y, bh, pol);
+                        if (!pre)
+                            tma_load_4d_pol(st + ST_Q + r * 128, &p.tm_q, &bar_full[s], 0, x, y, bh, pol_once);
+                    }
                 }
-                *reinterpret_cast<uint4 *>(sKh + sw128(p2, r8)) = pack8<T>(kh0);
-                *reinterpret_cast<uint4 *>(sKh + sw128(p2 + 1, r8)) = pack8<T>(kh1);
+            }
+        }
+        // no copy may still be landing when the CTA exits (after an abort the
+        // consumers may not have waited for them): bounded wait on the last
+        // issued phase of every stage
+        if (lane == 0) {
+            for (int it = (n_items > kStages ? n_items - kStages : 0); it < n_items; ++it) {
+                const int s = it % kStages;
+                if (issued & (1u << s)) mbar_wait(&bar_full[s], (it / kStages) & 1, 200000000ull);
+            }
+        }
+        __syncwarp();
+    } else if (warp == kWarpMma) {
+        // ---------------------------------------------------------- MMA issue
+        if (lane == 0) {
+            const uint32_t id_tf = idesc(2, 64, 64, 0, 0);     // tf32, both K-major
+            const uint32_t id_av = idesc(kFmt, 64, 64, 0, 1);  // A K-major, V as B (MN-major)
+            const uint32_t id_vk = idesc(kFmt, 64, 64, 1, 0);  // V^T as A (MN-major), K^ as B
+            const uint32_t sbase = smem_u32(sm);
+            auto dq = [&](uint32_t off) { return sdesc_sw128(sbase + off, 16, 1024); };
+            auto dv = [&](uint32_t off) { return sdesc_sw128(sbase + off, 8192, 1024); };
+            for (int it = 0; it < npre; ++it) {  // pre-pass: A_seg^T += V^T K^
+                const int s = it % kStages;
+                pwait(&bar_op[s], (it / kStages) & 1, &s_abort, p.err);
+                tc_fence_after_sync();
+                fence_proxy_async_smem();
+                const uint32_t so = s * ST_BYTES;
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_f16(tbase + TM_PRE, desc_add(dv(so + ST_V), ks * 2048),
+                            desc_add(dq(so + ST_KH), ks * 32), id_vk, (it > 0 || ks > 0) ? 1u : 0u);
+                mma_commit(&bar_empty[s]);
+            }
+            if (npre > 0) mma_commit(&bar_pre);
+            // chunk k: scores and dS^T (needs its operands)
+            auto issue_sc = [&](int k) {
+                const int it = npre + k, s = it % kStages;
+                pwait(&bar_op[s], (it / kStages) & 1, &s_abort, p.err);
+                tc_fence_after_sync();
+                fence_proxy_async_smem();
+                const uint32_t so = s * ST_BYTES, b = k & 1;
+                if (!sFlag[s]) {
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks) {
+                        const uint32_t o = (ks >> 2) * 8192 + (ks & 3) * 32;
+                        mma_tf32(tbase + TM_SC + 64 * b, desc_add(dq(so + ST_QH), o),
+                                 desc_add(dq(so + ST_KT), o), id_tf, ks > 0 ? 1u : 0u);
+                    }
+                }
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_f16(tbase + TM_DS + 64 * b, desc_add(dv(so + ST_V), ks * 2048),
+                            desc_add(dq(so + ST_KH), ks * 32), id_vk, ks > 0 ? 1u : 0u);
+                mma_commit(&bar_sc[b]);
+            };
+            if (L > 0) issue_sc(0);
+            for (int k = 0; k < L; ++k) {
+                const int it = npre + k, s = it % kStages;
+                const uint32_t so = s * ST_BYTES, b = k & 1;
+                // state k (input of chunk k) is in SB[b]; chunk k-1's dS^T has been consumed
+                pwait(&bar_s[b], (k >> 1) & 1, &s_abort, p.err);
+                if (k + 1 < L) issue_sc(k + 1);
+                pwait(&bar_a[b], (k >> 1) & 1, &s_abort, p.err);
+                tc_fence_after_sync();
+                fence_proxy_async_smem();
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {  // o = Q^ S_in
+                    const uint32_t o = (ks >> 2) * 8192 + (ks & 3) * 32;
+                    mma_tf32(tbase + TM_O + 64 * b, desc_add(dq(so + ST_QH), o),
+                             desc_add(dq(OFF_SB + 16384 * b), o), id_tf, ks > 0 ? 1u : 0u);
+                }
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)  // o += A V
+                    mma_f16(tbase + TM_O + 64 * b, desc_add(dq(OFF_A + 8192 * b), ks * 32),
+                            desc_add(dv(so + ST_V), ks * 2048), id_av, 1u);
+                mma_commit(&bar_o[b]);
+                mma_commit(&bar_empty[s]);
+            }
+            mma_commit(&bar_fin);
+            pwait(&bar_fin, 0, &s_abort, p.err);
+        }
+        __syncwarp();
+    } else if (warp < kWarpEpi0) {
+        // ------------------------------------------------------ operand warps
+        const int ow = warp - kWarpOp0;  // tokens 16 ow .. 16 ow + 15
+        const int p2 = 2 * lane;         // key dims p2, p2 + 1
+        const bool rev = p.dir & 1;      // token u sits in stage row 63 - u
+        const bool opl = (warp == kWarpOp0 && lane == 0);  // the group's polling thread
+        const int row0 = rev ? 63 - 16 * ow : 16 * ow;   // stage row of token 16 ow
+        const int rstep = rev ? -1 : 1;                   // stage-row step per token
+        // K^ (the K index of V^T K^ follows V's stage rows): this thread's 16
+        // tokens occupy the 16-byte chunks kc0, kc0 + 1 of rows p2, p2 + 1
+        const int kc0 = rev ? 6 - 2 * ow : 2 * ow;
+        auto store_kh = [&](uint8_t *kh, float *kh0, float *kh1) {
+            if (rev) {  // stage-row order is reversed token order
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const float t0 = kh0[j], t1 = kh1[j];
+                    kh0[j] = kh0[15 - j];
+                    kh0[15 - j] = t0;
+                    kh1[j] = kh1[15 - j];
+                    kh1[15 - j] = t1;
+                }
+            }
+            *reinterpret_cast<uint4 *>(kh + sw128(p2, kc0)) = pack8<T>(kh0);
+            *reinterpret_cast<uint4 *>(kh + sw128(p2, kc0 + 1)) = pack8<T>(kh0 + 8);
+            *reinterpret_cast<uint4 *>(kh + sw128(p2 + 1, kc0)) = pack8<T>(kh1);
+            *reinterpret_cast<uint4 *>(kh + sw128(p2 + 1, kc0 + 1)) = pack8<T>(kh1 + 8);
+        };
+        float2 gafter = make_float2(0.f, 0.f);
+        for (int it = 0; it < n_items; ++it) {
+            const int s = it % kStages;
+            const bool pre = it < npre;
+            const int k = it - npre;
+            gwait(opl, kBarOp, kOpThreads, &bar_full[s], (it / kStages) & 1, &s_abort, p.err);
+            uint8_t *st = sm + s * ST_BYTES;
+            const int len = sLen[s];
+            // 1. this thread's gates, q and k (everything is read before the
+            //    in-place overwrites below)
+            //    Loads are unconditional (every stage row is valid memory) and
+            //    tokens past the end are zeroed afterwards: no branch between
+            //    the loads, so they are all in flight at once.
+            float2 a[16];
+            uint32_t qw[16], kw[16];
+            float2 l = make_float2(0.f, 0.f);
+            const int nin = len - 16 * ow;  // this thread's tokens kk < nin are real
+            {
+                const float *lr = reinterpret_cast<const float *>(st + ST_LA) + row0 * 64 + p2;
+                const uint8_t *kr = st + ST_K + row0 * 128 + p2 * 2;
+                const uint8_t *qr = st + ST_Q + row0 * 128 + p2 * 2;
+                float2 x[16];
+#pragma unroll
+                for (int kk = 0; kk < 16; ++kk) {
+                    x[kk] = ld2(lr + kk * rstep * 64);
+                    kw[kk] = *reinterpret_cast<const uint32_t *>(kr + kk * rstep * 128);
+                    qw[kk] = *reinterpret_cast<const uint32_t *>(qr + kk * rstep * 128);
+                }
+#pragma unroll
+                for (int kk = 0; kk < 16; ++kk) {
+                    const bool in = kk < nin;
+                    x[kk] = in ? x[kk] : make_float2(0.f, 0.f);
+                    kw[kk] = in ? kw[kk] : 0u;
+                    qw[kk] = in ? qw[kk] : 0u;
+                    l.x += x[kk].x;
+                    l.y += x[kk].y;
+                    a[kk] = ex2_2(x[kk]);
+                }
+            }
+            float *tot = sTot + (it & 1) * 256;
+            st2(tot + ow * 64 + p2, l);
+            named_bar_sync(kBarOp, kOpThreads);
+            // 2. where this thread's rows sit in the chunk
+            float2 before = make_float2(0.f, 0.f), g = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int o = 0; o < 4; ++o) {
+                const float2 t = ld2(tot + o * 64 + p2);
+                if (o < ow) {
+                    before.x += t.x;
+                    before.y += t.y;
+                }
+                g.x += t.x;
+                g.y += t.y;
+            }
+            const float2 after = make_float2(g.x - before.x - l.x, g.y - before.y - l.y);
+            if (pre) {
+                // K^ relative to the segment end: k . e^{G_after + (gates after u in the chunk)}
+                float2 f = ex2_2(make_float2(gafter.x + after.x, gafter.y + after.y));
+                float kh0[16], kh1[16];
+#pragma unroll
+                for (int kk = 15; kk >= 0; --kk) {
+                    const float2 kv = Pack2<T>::unpack(kw[kk]);
+                    const float2 h = fmul2(kv, f);
+                    kh0[kk] = h.x;
+                    kh1[kk] = h.y;
+                    f = fmul2(f, a[kk]);
+                }
+                store_kh(st + ST_KH, kh0, kh1);
+                gafter.x += g.x;
+                gafter.y += g.y;
+                if (it == npre - 1) {  // the segment's gate totals
+                    if (ow == 0) st2(p.aggg + slot * 64 + p2, gafter);
+                    __threadfence();
+                    mbar_arrive(&bar_owpre);
+                }
+            } else {
+                const bool unsafe = __any_sync(0xffffffffu, (-g.x > kSpanLimit) || (-g.y > kSpanLimit));
+                if (unsafe) {
+                    // exact scores: b (log2 domain) in place of log_alpha, then
+                    // A[t,s] = sum_i q_ti k_si 2^{b_ti - b_si} for s <= t
+                    float2 cb = before;
+                    float *lat = reinterpret_cast<float *>(st + ST_LA);
+#pragma unroll
+                    for (int kk = 0; kk < 16; ++kk) {
+                        const int u = 16 * ow + kk, pr = rev ? 63 - u : u;
+                        const float2 x = (u < len) ? ld2(lat + pr * 64 + p2) : make_float2(0.f, 0.f);
+                        cb.x += x.x;
+                        cb.y += x.y;
+                        st2(lat + pr * 64 + p2, make_float2(cb.x * kLog2e, cb.y * kLog2e));
+                    }
+                    named_bar_sync(kBarOp, kOpThreads);
+                    if (k >= 2) gwait(opl, kBarOp, kOpThreads, &bar_a[k & 1], ((k >> 1) - 1) & 1, &s_abort, p.err);
+                    const int qd = warp & 3, r0 = 16 * qd + (lane >> 2), cq = 2 * (lane & 3);
+                    uint32_t sc[32];
+#pragma unroll 1
+                    for (int e = 0; e < 32; ++e) {
+                        const int t = r0 + 8 * ((e >> 1) & 1), sx = 8 * (e >> 2) + cq + (e & 1);
+                        float acc = 0.f;
+                        if (sx <= t && t < len) {
+                            const int pt = rev ? 63 - t : t, ps = rev ? 63 - sx : sx;
+                            const T *qr = reinterpret_cast<const T *>(st + ST_Q + pt * 128);
+                            const T *kr = reinterpret_cast<const T *>(st + ST_K + ps * 128);
+                            for (int i = 0; i < FD; ++i)
+                                acc = fmaf(to_f32(qr[i]) * to_f32(kr[i]),
+                                           fast_exp2(lat[pt * 64 + i] - lat[ps * 64 + i]), acc);
+                        }
+                        sc[e] = __float_as_uint(acc);
+                    }
+                    tmem_st16x256(tbase + TM_SC + 64 * (k & 1) + ((uint32_t)(32 * qd) << 16), sc);
+                    tmem_st_wait();
+                    named_bar_sync(kBarOp, kOpThreads);  // b is no longer read: Q^ may overwrite it
+                }
+                // Q^ = q . e^{b_u} (running product of the alphas up to u)
+                float2 e = ex2_2(before);
+                uint8_t *qh = st + ST_QH;
+#pragma unroll
+                for (int kk = 0; kk < 16; ++kk) {
+                    const int u = 16 * ow + kk;
+                    e = fmul2(e, a[kk]);
+                    const float2 v = fmul2(Pack2<T>::unpack(qw[kk]), e);
+                    *reinterpret_cast<uint2 *>(qh + tf32_kmaj(u, p2)) = make_uint2(tf32_rn(v.x), tf32_rn(v.y));
+                }
+                // K^ = k . e^{g - b_u} (product of the alphas after u), K~ = K^ . e^{-g}
+                float2 f = ex2_2(after);
+                const float2 m = unsafe ? make_float2(0.f, 0.f) : ex2_2(make_float2(-g.x, -g.y));
+                uint8_t *kt = st + ST_KT;
+                float kh0[16], kh1[16];
+#pragma unroll
+                for (int kk = 15; kk >= 0; --kk) {
+                    const int u = 16 * ow + kk;
+                    const float2 h = fmul2(Pack2<T>::unpack(kw[kk]), f);
+                    kh0[kk] = h.x;
+                    kh1[kk] = h.y;
+                    const float2 t2 = fmul2(h, m);
+                    *reinterpret_cast<uint2 *>(kt + tf32_kmaj(u, p2)) = make_uint2(tf32_rn(t2.x), tf32_rn(t2.y));
+                    f = fmul2(f, a[kk]);
+                }
+                store_kh(st + ST_KH, kh0, kh1);
+                if (ow == 0) {
+                    st2(sGam + s * 64 + p2, ex2_2(g));
+                    if (lane == 0) sFlag[s] = unsafe ? 1 : 0;
+                }
             }
             fence_proxy_async_smem();
             tc_fence_before_sync();
-            __syncthreads();
-            tc_fence_after_sync();
-            if (r8 == 7) {  // the last row group holds the chunk totals of columns p2, p2+1
-                float2 ga = *reinterpret_cast<float2 *>(sGa + p2);
-                ga.x += G.g0;
-                ga.y += G.g1;
-                *reinterpret_cast<float2 *>(sGa + p2) = ga;
-            }
-            if (tid == 0) {
-                fence_proxy_async_smem();  // v landed by cp.async, observed by this thread
-                const uint64_t vd = sdesc_sw128(smem_u32(vt), 8192, 1024);
-                const uint64_t kd = sdesc_sw128(smem_u32(sKh), 16, 1024);
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_f16(tbase + TM_DS, desc_add(vd, ks * 2048), desc_add(kd, ks * 32), id_vk,
-                            (idx > 0 || ks > 0) ? 1u : 0u);
-                mma_commit(&bar_mma);
-            }
-            if (idx + 2 < nl) fill_rows(p, bh, c - 2, sRow + 64 * st);
-            ok = cta_wait(&bar_mma, ph_mma, ok, &s_ok);
-            ph_mma ^= 1;
-            tc_fence_after_sync();
-            if (idx + 2 < nl) {  // this stage is free again: fetch chunk c - 2 into it
-                const int *rows = sRow + 64 * st;
-                copy_tile16(st ? sm + OFF_K1 : sK, p.k, rows);
-                copy_tile32(st ? sm + OFF_LA1 : sm + OFF_LA, p.la, rows);
-                copy_tile16(st ? sm + OFF_V1 : sV, p.v, rows);
-                cp_async_arrive(&bar_st[st]);
-            }
+            mbar_arrive(&bar_op[s]);
         }
-        // publish the aggregate A_seg^T ([j][i]) and the gate totals
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            uint32_t r[16];
-            const int cb = 32 * ch + 16 * hh;
-            tmem_ld16(tbase + TM_DS + lane_off + cb, r);
-            tmem_ld_wait();
-            if (act) {
-                const size_t off = slot * 4096 + row16 * 64 + cb;
-#pragma unroll
-                for (int e = 0; e < 16; e += 4) {
-                    const float4 v4 = make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]),
-                                                  __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
-                    *reinterpret_cast<float4 *>(p.agg + off + e) = v4;
-                }
-            }
-        }
-        if (tid < 64) p.aggg[slot * 64 + tid] = sGa[tid];
-        __threadfence();
-        tc_fence_before_sync();
-        __syncthreads();
-        tc_fence_after_sync();
-        if (tid == 0) st_release(p.flag + slot, 1);
-    }
-
-    // first main-pass chunk: its loads overlap the boundary pass
-    fill_rows(p, bh, c_begin, sRow + 64 * (c_begin & 1));
-    __syncthreads();
-    {
-        const int *rows = sRow + 64 * (c_begin & 1);
-        copy_tile16(sQ, p.q, rows);
-        copy_tile16(sK, p.k, rows);
-        copy_tile32(reinterpret_cast<uint8_t *>(sLA), p.la, rows);
-        cp_async_arrive(&bar_ld);
-        copy_tile16(sV, p.v, rows);
-        cp_async_arrive(&bar_v);
-    }
-
-    // -------------------------------------------------------- boundary pass
-    // S_in^T (fp32, [j][i] row-major) is assembled in the A/K^ tiles' space.
-    float *sSin = reinterpret_cast<float *>(sA);
-    if (seg > 0) {
-        // 1. every earlier segment of this (b,h) must have published its
-        //    aggregate (bounded waits, one lane per predecessor)
-        if (warp == 0) {
-            int fail = 0;
-            for (int j = lane; j < seg; j += 32)
-                if (wait_flag(p.flag + (size_t)bh * p.P + j, p.err) == 0) fail = 1;
-            fail = __any_sync(0xffffffffu, fail);
-            if (lane == 0) s_fail = fail;
-        }
-        __syncthreads();
-        const int nfold = seg;
-        if (s_fail) ok = false;
-        // 2. per key dim i: scale of the term of segment seg-1-d, e^{sum of the
-        //    log gates of the d segments between it and this one} (in QH's space)
-        float *sAg = reinterpret_cast<float *>(sQH);  // [nfold][64], nfold < kMaxSegments
-        for (int e = tid; e < nfold * 64; e += kThreads)
-            sAg[e] = __ldcg(p.aggg + ((size_t)bh * p.P + (seg - 1 - (e >> 6))) * 64 + (e & 63));
-        __syncthreads();
-        if (tid < 64) {
-            float acc = 0.f;
-            for (int d = 0; d < nfold; ++d) {
-                const float a = sAg[d * 64 + tid];
-                sAg[d * 64 + tid] = fast_exp2(acc * kLog2e);
-                acc += a;
-            }
-        }
-        __syncthreads();
-        // 3. fold, nearest segment first (a fixed order: the result does not
-        //    depend on timing): thread -> (row j, 16 columns i)
-        {
-            const int j = tid >> 2, c0 = 16 * (tid & 3);
-            float acc[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) acc[e] = 0.f;
-            // the loads of kFoldBatch aggregates are all issued before any of
-            // them is consumed, so several L2 round trips overlap
-            constexpr int kFoldBatch = 4;
-            const float *base = p.agg + (size_t)bh * p.P * 4096 + j * 64 + c0;
-            for (int d0 = 0; d0 < nfold; d0 += kFoldBatch) {
-                float4 v[kFoldBatch][4];
-#pragma unroll
-                for (int b = 0; b < kFoldBatch; ++b) {
-                    const int d = min(d0 + b, nfold - 1);
-                    const float *src = base + (size_t)(seg - 1 - d) * 4096;
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) v[b][q] = __ldcg(reinterpret_cast<const float4 *>(src + 4 * q));
-                }
-#pragma unroll
-                for (int b = 0; b < kFoldBatch; ++b) {
-                    if (d0 + b < nfold) {
-                        const float *sc = sAg + (d0 + b) * 64 + c0;
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const float4 s4 = *reinterpret_cast<const float4 *>(sc + 4 * q);
-                            acc[4 * q] = fmaf(s4.x, v[b][q].x, acc[4 * q]);
-                            acc[4 * q + 1] = fmaf(s4.y, v[b][q].y, acc[4 * q + 1]);
-                            acc[4 * q + 2] = fmaf(s4.z, v[b][q].z, acc[4 * q + 2]);
-                            acc[4 * q + 3] = fmaf(s4.w, v[b][q].w, acc[4 * q + 3]);
-                        }
-                    }
-                }
-            }
-#pragma unroll
-            for (int q4 = 0; q4 < 16; q4 += 4)
-                *reinterpret_cast<float4 *>(sSin + j * 64 + c0 + q4) =
-                    make_float4(acc[q4], acc[q4 + 1], acc[q4 + 2], acc[q4 + 3]);
-        }
-        __syncthreads();
     } else {
-        for (int e = tid; e < 4096; e += kThreads) sSin[e] = 0.f;
-        __syncthreads();
-    }
-    // S_in^T -> TMEM state and the tf32 operand (rows j, K = i)
-    {
+        // ----------------------------------------------------- epilogue warps
+        const int qd = warp & 3;                       // TMEM lane quadrant
+        const uint32_t lo = (uint32_t)(32 * qd) << 16;
+        const int r0 = 16 * qd + (lane >> 2);          // rows r0 and r0 + 8
+        const int cq = 2 * (lane & 3);                 // columns 8 c + cq + {0, 1}
+        const bool rev = p.dir & 1;
+        const bool epl = (warp == kWarpEpi0 && lane == 0);  // the group's polling thread
+        bool ok = true;
+        float S[32];  // S^T[j][i]: j = r0 + 8 ((x >> 1) & 1), i = 8 (x >> 2) + cq + (x & 1)
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            const int cb = 32 * ch + 16 * hh;
-            uint32_t r[16];
-            const float *src = sSin + row16 * 64 + cb;
-#pragma unroll
-            for (int e = 0; e < 16; e += 4) {
-                const float4 v4 = act ? *reinterpret_cast<const float4 *>(src + e) : make_float4(0.f, 0.f, 0.f, 0.f);
-                r[e] = __float_as_uint(v4.x);
-                r[e + 1] = __float_as_uint(v4.y);
-                r[e + 2] = __float_as_uint(v4.z);
-                r[e + 3] = __float_as_uint(v4.w);
-            }
-            tmem_st16(tbase + TM_S + lane_off + cb, r);
-            if (act) {
-#pragma unroll
-                for (int e = 0; e < 16; e += 4)
-                    *reinterpret_cast<uint4 *>(sB1 + tf32_kmaj<128>(64 + row16, cb + e)) =
-                        make_uint4(tf32_round(__uint_as_float(r[e])), tf32_round(__uint_as_float(r[e + 1])),
-                                   tf32_round(__uint_as_float(r[e + 2])), tf32_round(__uint_as_float(r[e + 3])));
-            }
-        }
-        tmem_st_wait();
-        fence_proxy_async_smem();
-        tc_fence_before_sync();
-        __syncthreads();
-        tc_fence_after_sync();
-    }
+        for (int x = 0; x < 32; ++x) S[x] = 0.f;
 
-    // ------------------------------------------------------------ main pass
-    for (int c = c_begin; c < c_end; ++c) {
-        const int len = min(FC, p.n - c * FC);
-        const int *rows = sRow + 64 * (c & 1);
-        int *rows_next = sRow + 64 * ((c + 1) & 1);
-        const bool more = c + 1 < c_end;
-        if (c == c_begin) {  // later chunks wait for their q,k,log_alpha at the end of the previous one
-            ok = cta_wait(&bar_ld, ph_ld, ok, &s_ok);
-            ph_ld ^= 1;
-        }
-        // ---- gate factors and operands
-        GateRows G;
-        gate_rows(sLA, sTot, p2, r8, len, G);
-        if (r8 == 7)
-            *reinterpret_cast<float2 *>(sGam + p2) =
-                make_float2(fast_exp2(G.g0 * kLog2e), fast_exp2(G.g1 * kLog2e));
-        if (more) fill_rows(p, bh, c + 1, rows_next);
-        const bool my_unsafe = (-G.g0 > kSpanLimit) || (-G.g1 > kSpanLimit);
-        {
-            // Q^ = q . e^{b_u}: running product of the alphas up to u
-            float e0 = fast_exp2(G.pre0 * kLog2e), e1 = fast_exp2(G.pre1 * kLog2e);
+        if (npre > 0) {  // publish the aggregate A_seg^T and raise this segment's flag
+            ok = gwait(epl, kBarEpi, kEpiThreads, &bar_pre, 0, &s_abort, p.err, 256) && ok;
+            tc_fence_after_sync();
+            uint32_t r[32];
+            tmem_ld16x256(tbase + TM_PRE + lo, r);
+            tmem_ld_wait();
+            float *dst = p.agg + slot * 4096;
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const int u = 8 * r8 + k;
-                float2 qv = make_float2(0.f, 0.f);
-                if (u < len)
-                    qv = Pack2<T>::unpack(
-                        *reinterpret_cast<const uint32_t *>(sQ + sw128(u, p2 >> 3) + (p2 & 7) * 2));
-                e0 *= G.a0[k];
-                e1 *= G.a1[k];
-                *reinterpret_cast<uint2 *>(sQH + tf32_kmaj<64>(u, p2)) =
-                    make_uint2(tf32_round(qv.x * e0), tf32_round(qv.y * e1));
+            for (int x = 0; x < 32; x += 2) {
+                const int j = r0 + 8 * ((x >> 1) & 1), i = 8 * (x >> 2) + cq;
+                st2(dst + j * 64 + i, make_float2(__uint_as_float(r[x]), __uint_as_float(r[x + 1])));
             }
-            // K^ = k . e^{g - b_u} (product of the alphas after u), K~ = K^ . e^{-g}
-            float f0 = fast_exp2(G.suf0 * kLog2e), f1 = fast_exp2(G.suf1 * kLog2e);
-            const float m0 = my_unsafe ? 0.f : fast_exp2(-G.g0 * kLog2e);
-            const float m1 = my_unsafe ? 0.f : fast_exp2(-G.g1 * kLog2e);
-            float kh0[8], kh1[8];
-#pragma unroll
-            for (int k = 7; k >= 0; --k) {
-                const int u = 8 * r8 + k;
-                float2 kv = make_float2(0.f, 0.f);
-                if (u < len)
-                    kv = Pack2<T>::unpack(
-                        *reinterpret_cast<const uint32_t *>(sK + sw128(u, p2 >> 3) + (p2 & 7) * 2));
-                kh0[k] = kv.x * f0;
-                kh1[k] = kv.y * f1;
-                *reinterpret_cast<uint2 *>(sB1 + tf32_kmaj<128>(u, p2)) =
-                    make_uint2(tf32_round(kh0[k] * m0), tf32_round(kh1[k] * m1));
-                f0 *= G.a0[k];
-                f1 *= G.a1[k];
-            }
-            *reinterpret_cast<uint4 *>(sKh + sw128(p2, r8)) = pack8<T>(kh0);
-            *reinterpret_cast<uint4 *>(sKh + sw128(p2 + 1, r8)) = pack8<T>(kh1);
+            ok = gwait(epl, kBarEpi, kEpiThreads, &bar_owpre, 0, &s_abort, p.err) && ok;
+            __threadfence();
+            named_bar_sync(kBarEpi, kEpiThreads);
+            if (warp == kWarpEpi0 && lane == 0 && ok) st_release(p.flag + slot, 1);
         }
-        fence_proxy_async_smem();
-        tc_fence_before_sync();
-        const int unsafe = __syncthreads_or(my_unsafe);
-        tc_fence_after_sync();
-        if (tid == 0) {  // [scores | o] = Q^ [K~ ; S_in^T]^T
-            const uint64_t ad = sdesc_sw128(smem_u32(sQH), 16, 1024);
-            const uint64_t bd = sdesc_sw128(smem_u32(sB1), 16, 1024);
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-                mma_tf32(tbase + TM_RAW, desc_add(ad, (ks >> 2) * 8192 + (ks & 3) * 32),
-                         desc_add(bd, (ks >> 2) * 16384 + (ks & 3) * 32), id_tf, ks > 0 ? 1u : 0u);
-            mma_commit(&bar_mma);
-        }
-        if (unsafe) {
-            // the exact score path needs b (log2 domain) of every row: keep it in sLA
-            float c0 = G.pre0, c1 = G.pre1;
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const int u = 8 * r8 + k;
-                float2 *pl = reinterpret_cast<float2 *>(sLA + u * 64 + p2);
-                if (u < len) {
-                    const float2 x = *pl;
-                    c0 += x.x;
-                    c1 += x.y;
+        if (seg > 0) {  // fold the earlier segments' aggregates, nearest first
+            if (warp == kWarpEpi0) {
+                bool got = true;
+                for (int j = lane; j < seg; j += 32) got = wait_flag(p.flag + (size_t)bh * p.P + j) && got;
+                if (!__all_sync(0xffffffffu, got) && lane == 0) {
+                    s_abort = 1;
+                    latch_error(p.err, kDevErrTimeout);
                 }
-                *pl = make_float2(c0 * kLog2e, c1 * kLog2e);
             }
-        } else if (more) {
-            copy_tile16(sQ, p.q, rows_next);
-            copy_tile16(sK, p.k, rows_next);
-            copy_tile32(reinterpret_cast<uint8_t *>(sLA), p.la, rows_next);
-            cp_async_arrive(&bar_ld);
-        }
-        ok = cta_wait(&bar_mma, ph_mma, ok, &s_ok);
-        ph_mma ^= 1;
-        tc_fence_after_sync();
-        // ---- causal mask of the scores -> A (rows t, K = s)
-        if (!unsafe) {
+            named_bar_sync(kBarEpi, kEpiThreads);
+            if (s_abort) ok = false;
+            float2 acc[8];  // log-gate sums of the segments between the source and this one
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                uint32_t r[16];
-                tmem_ld16(tbase + TM_RAW + lane_off + 32 * ch + 16 * hh, r);
-                tmem_ld_wait();
-                if (act) {
-                    const int t = row16;
-                    float a[16];
+            for (int c = 0; c < 8; ++c) acc[c] = make_float2(0.f, 0.f);
+            // software-pipelined: the next aggregate's loads are in flight
+            // while the current one is folded
+            float2 v[16], gt[8], vn[16], gtn[8];
+            auto load = [&](int d, float2 *vv, float2 *gg) {
+                const size_t src = (size_t)bh * p.P + (seg - 1 - d);
+                const float *ag = p.agg + src * 4096;
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int s = 32 * ch + 16 * hh + e;
-                        a[e] = (s <= t) ? __uint_as_float(r[e]) : 0.f;
+                for (int x = 0; x < 32; x += 2) {
+                    const int j = r0 + 8 * ((x >> 1) & 1), i = 8 * (x >> 2) + cq;
+                    vv[x >> 1] = __ldcg(reinterpret_cast<const float2 *>(ag + j * 64 + i));
+                }
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    gg[c] = __ldcg(reinterpret_cast<const float2 *>(p.aggg + src * 64 + 8 * c + cq));
+            };
+            if (ok) load(0, v, gt);
+            for (int d = 0; d < seg && ok; ++d) {
+                if (d + 1 < seg) load(d + 1, vn, gtn);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const float2 sc = ex2_2(acc[c]);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int x = 4 * c + 2 * h;
+                        const float2 t = ffma2(sc, v[x >> 1], make_float2(S[x], S[x + 1]));
+                        S[x] = t.x;
+                        S[x + 1] = t.y;
                     }
-                    *reinterpret_cast<uint4 *>(sA + sw128(t, 4 * ch + 2 * hh)) = pack8<T>(a);
-                    *reinterpret_cast<uint4 *>(sA + sw128(t, 4 * ch + 2 * hh + 1)) = pack8<T>(a + 8);
+                    acc[c].x += gt[c].x;
+                    acc[c].y += gt[c].y;
                 }
-            }
-        } else {
-            __syncthreads();  // b of every row is in sLA
-            // exact scores A[t,s] = sum_i q_ti k_si 2^{b_ti - b_si}, s <= t (every factor <= 1)
-            const int t = tid >> 2, s0 = 16 * (tid & 3);
-            float a[16];
-#pragma unroll 1
-            for (int e = 0; e < 16; ++e) {
-                const int s = s0 + e;
-                float acc = 0.f;
-                if (s <= t && t < len) {
-                    for (int i = 0; i < FD; ++i)
-                        acc = fmaf(tile16<T>(sQ, t, i) * tile16<T>(sK, s, i),
-                                   fast_exp2(sLA[t * 64 + i] - sLA[s * 64 + i]), acc);
-                }
-                a[e] = acc;
-            }
-            *reinterpret_cast<uint4 *>(sA + sw128(t, s0 >> 3)) = pack8<T>(a);
-            *reinterpret_cast<uint4 *>(sA + sw128(t, (s0 >> 3) + 1)) = pack8<T>(a + 8);
-        }
-        fence_proxy_async_smem();
-        tc_fence_before_sync();
-        ok = cta_wait(&bar_v, ph_v, ok, &s_ok);  // also publishes the A rows
-        ph_v ^= 1;
-        tc_fence_after_sync();
-        if (unsafe && more) {
-            copy_tile16(sQ, p.q, rows_next);
-            copy_tile16(sK, p.k, rows_next);
-            copy_tile32(reinterpret_cast<uint8_t *>(sLA), p.la, rows_next);
-            cp_async_arrive(&bar_ld);
-        }
-        if (tid == 0) {
-            fence_proxy_async_smem();  // v landed by cp.async, observed by this thread
-            const uint64_t ad = sdesc_sw128(smem_u32(sA), 16, 1024);
-            const uint64_t vd = sdesc_sw128(smem_u32(sV), 8192, 1024);
-            const uint64_t kd = sdesc_sw128(smem_u32(sKh), 16, 1024);
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {  // o += A V ;  dS^T = V^T K^
-                const uint64_t v = desc_add(vd, ks * 2048);
-                mma_f16(tbase + TM_O, desc_add(ad, ks * 32), v, id_av, 1u);
-                mma_f16(tbase + TM_DS, v, desc_add(kd, ks * 32), id_vk, ks > 0 ? 1u : 0u);
-            }
-            mma_commit(&bar_mma);
-        }
-        ok = cta_wait(&bar_mma, ph_mma, ok, &s_ok);
-        ph_mma ^= 1;
-        tc_fence_after_sync();
-        // ---- outputs and the state update (rows t / rows j of lanes 0..15)
+                for (int x = 0; x < 16; ++x) v[x] = vn[x];
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            const int cb = 32 * ch + 16 * hh;
-            const uint32_t col = lane_off + cb;
-            uint32_t ro[16], rs[16], rd[16];
-            tmem_ld16(tbase + TM_O + col, ro);
-            tmem_ld16(tbase + TM_S + col, rs);
-            tmem_ld16(tbase + TM_DS + col, rd);
-            tmem_ld_wait();
-            if (act && row16 < len) {
-                uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<T *>(p.out) +
-                                                       (size_t)rows[row16] * FD + cb);
-                float o[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) o[e] = __uint_as_float(ro[e]);
-                dst[0] = pack8<T>(o);
-                dst[1] = pack8<T>(o + 8);
-            }
-            // S^T[j][i] <- e^{g_i} S^T[j][i] + dS^T[j][i]
-#pragma unroll
-            for (int e = 0; e < 16; e += 4) {
-                const float4 g4 = *reinterpret_cast<const float4 *>(sGam + cb + e);
-                rs[e] = __float_as_uint(fmaf(g4.x, __uint_as_float(rs[e]), __uint_as_float(rd[e])));
-                rs[e + 1] = __float_as_uint(fmaf(g4.y, __uint_as_float(rs[e + 1]), __uint_as_float(rd[e + 1])));
-                rs[e + 2] = __float_as_uint(fmaf(g4.z, __uint_as_float(rs[e + 2]), __uint_as_float(rd[e + 2])));
-                rs[e + 3] = __float_as_uint(fmaf(g4.w, __uint_as_float(rs[e + 3]), __uint_as_float(rd[e + 3])));
-            }
-            tmem_st16(tbase + TM_S + col, rs);
-            if (act && more) {
-#pragma unroll
-                for (int e = 0; e < 16; e += 4)
-                    *reinterpret_cast<uint4 *>(sB1 + tf32_kmaj<128>(64 + row16, cb + e)) =
-                        make_uint4(tf32_round(__uint_as_float(rs[e])), tf32_round(__uint_as_float(rs[e + 1])),
-                                   tf32_round(__uint_as_float(rs[e + 2])), tf32_round(__uint_as_float(rs[e + 3])));
+                for (int c = 0; c < 8; ++c) gt[c] = gtn[c];
             }
         }
-        tmem_st_wait();
-        fence_proxy_async_smem();
-        tc_fence_before_sync();
-        if (more) {  // the next chunk's q,k,log_alpha; the barrier also ends this epilogue
-            ok = cta_wait(&bar_ld, ph_ld, ok, &s_ok);
-            ph_ld ^= 1;
-        } else {
-            __syncthreads();
-        }
-        tc_fence_after_sync();
-        if (more) {
-            copy_tile16(sV, p.v, rows_next);
-            cp_async_arrive(&bar_v);
-        }
-    }
+        // state 0 (the incoming state) -> SB[0]
+        auto store_state = [&](int b) {
+            uint8_t *sb = sm + OFF_SB + 16384 * b;
+#pragma unroll
+            for (int x = 0; x < 32; x += 2) {
+                const int j = r0 + 8 * ((x >> 1) & 1), i = 8 * (x >> 2) + cq;
+                *reinterpret_cast<uint2 *>(sb + tf32_kmaj(j, i)) = make_uint2(tf32_rn(S[x]), tf32_rn(S[x + 1]));
+            }
+            fence_proxy_async_smem();
+        };
+        store_state(0);
+        mbar_arrive(&bar_s[0]);
 
-    if (seg == p.P - 1 && p.final_state) {  // S^T rows -> smem -> final_state rows i
-        float *sFs = reinterpret_cast<float *>(sQH);  // [64][65], inside the idle Q^/K~ tiles
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            uint32_t rs[16];
-            const int cb = 32 * ch + 16 * hh;
-            tmem_ld16(tbase + TM_S + lane_off + cb, rs);
+        // output of chunk kp (its o is complete once bar_o says so)
+        int prow[2] = {0, 0}, plen = 0;
+        auto emit = [&](int kp) {
+            const int b = kp & 1;
+            ok = gwait(epl, kBarEpi, kEpiThreads, &bar_o[b], (kp >> 1) & 1, &s_abort, p.err) && ok;
+            tc_fence_after_sync();
+            uint32_t r[32];
+            tmem_ld16x256(tbase + TM_O + 64 * b + lo, r);
             tmem_ld_wait();
-            if (act) {
+            if (ok) {
 #pragma unroll
-                for (int e = 0; e < 16; ++e) sFs[(cb + e) * 65 + row16] = __uint_as_float(rs[e]);
+                for (int h = 0; h < 2; ++h) {
+                    if (r0 + 8 * h < plen) {
+                        uint32_t *dst = reinterpret_cast<uint32_t *>(reinterpret_cast<T *>(p.out) +
+                                                                     (size_t)prow[h] * FD + cq);
+#pragma unroll
+                        for (int c = 0; c < 8; ++c)
+                            dst[4 * c] = Pack2<T>::pack(__uint_as_float(r[4 * c + 2 * h]),
+                                                        __uint_as_float(r[4 * c + 2 * h + 1]));
+                    }
+                }
+            }
+        };
+
+        uint8_t *const sAbuf = sm + OFF_A;
+        for (int k = 0; k < L; ++k) {
+            const int it = npre + k, s = it % kStages, b = k & 1;
+            // the operand warps' release of this stage makes its row table,
+            // length and gate factors visible here
+            ok = gwait(epl, kBarEpi, kEpiThreads, &bar_op[s], (it / kStages) & 1, &s_abort, p.err) && ok;
+            ok = gwait(epl, kBarEpi, kEpiThreads, &bar_sc[b], (k >> 1) & 1, &s_abort, p.err) && ok;
+            tc_fence_after_sync();
+            // stage-local values, read before the stage can be recycled
+            const int *rows = sRows + s * 64;
+            const int len = sLen[s];
+            const int row0 = rows[r0], row1 = rows[r0 + 8];
+            float2 gam[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) gam[c] = ld2(sGam + s * 64 + 8 * c + cq);
+            // causal mask of the scores -> A[b] (rows t, K = s)
+            {
+                uint32_t r[32];
+                tmem_ld16x256(tbase + TM_SC + 64 * b + lo, r);
+                tmem_ld_wait();
+                uint8_t *sa = sAbuf + 8192 * b;
+                // columns follow V's stage rows: token s at column s, or 63 - s
+                // for reversed scans
+                // (column 63 - s = 16-byte chunk 7 ^ c, element 6 ^ cq, the pair swapped)
+                const int cx = rev ? 7 : 0, ex = rev ? 6 : 0;
+#pragma unroll
+                for (int x = 0; x < 32; x += 2) {
+                    const int t = r0 + 8 * ((x >> 1) & 1), sx = 8 * (x >> 2) + cq;
+                    const float v0 = (sx <= t) ? __uint_as_float(r[x]) : 0.f;
+                    const float v1 = (sx + 1 <= t) ? __uint_as_float(r[x + 1]) : 0.f;
+                    *reinterpret_cast<uint32_t *>(sa + sw128(t, (x >> 2) ^ cx) + (cq ^ ex) * 2) =
+                        rev ? Pack2<T>::pack(v1, v0) : Pack2<T>::pack(v0, v1);
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before_sync();
+            mbar_arrive(&bar_a[b]);
+            if (k > 0) emit(k - 1);  // chunk k-1's product is done: SB[(k+1)&1] is free again
+            prow[0] = row0;
+            prow[1] = row1;
+            plen = len;
+            // state update S_{k+1} = diag(e^{g}) S_k + dS_k  (S^T: scale column i)
+            {
+                uint32_t r[32];
+                tmem_ld16x256(tbase + TM_DS + 64 * b + lo, r);
+                tmem_ld_wait();
+#pragma unroll
+                for (int x = 0; x < 32; x += 2) {
+                    const float2 t = ffma2(gam[x >> 2], make_float2(S[x], S[x + 1]),
+                                           make_float2(__uint_as_float(r[x]), __uint_as_float(r[x + 1])));
+                    S[x] = t.x;
+                    S[x + 1] = t.y;
+                }
+            }
+            if (k + 1 < L) store_state((k + 1) & 1);
+            tc_fence_before_sync();
+            mbar_arrive(&bar_s[(k + 1) & 1]);
+        }
+        if (L > 0) emit(L - 1);
+        if (seg == p.P - 1 && p.final_state && ok) {
+            float *fs = p.final_state + (size_t)bh * 4096;
+#pragma unroll
+            for (int x = 0; x < 32; ++x) {
+                const int j = r0 + 8 * ((x >> 1) & 1), i = 8 * (x >> 2) + cq + (x & 1);
+                fs[i * 64 + j] = S[x];
             }
         }
-        __syncthreads();
-        for (int e = tid; e < 4096; e += kThreads)
-            p.final_state[(size_t)bh * 4096 + e] = sFs[(e >> 6) * 65 + (e & 63)];
     }
-        if (!ok) latch_error(p.err, kDevErrTimeout);
 
     // ------------------------------------------------------------- teardown
     tc_fence_before_sync();
     __syncthreads();
-    if (warp == 1) tmem_dealloc(tbase, kTmemCols);
+    tc_fence_after_sync();
+    if (warp == kWarpMma) tmem_dealloc(tbase, kTmemCols);
     if (tid == 0) {
         __threadfence();
         const unsigned prev = atomicAdd(&p.ctr[1], 1u);
@@ -784,23 +818,39 @@ __global__ void __launch_bounds__(kThreads, 2) gla_fused_kernel(const __grid_con
     }
 }
 
-constexpr int kTargetCtas = 2 * 148;  // two resident CTAs on each of the B200's SMs
+constexpr int kSMs = 148;
 
 struct Plan {
     int nc, P, L;
 };
 
+// Segments per (b,h).  More segments put more SMs to work and shorten each
+// CTA's serial chain of chunks, but every segment except the last adds a
+// pre-pass over its chunks and every segment folds all earlier aggregates.
+// The choice minimises a time model built from this kernel's measured costs
+// on B200 (microseconds): a main-pass chunk, a pre-pass chunk, one folded
+// aggregate, and the fixed cost of publishing and waiting for flags; CTAs
+// beyond one per SM run in further waves.
 Plan make_plan(const Problem &pr) {
-    Plan pl;
-    pl.nc = (pr.n + FC - 1) / FC;
+    constexpr double kMain = 2.2, kPre = 1.2, kFold = 0.5, kFlag = 3.0;
+    Plan best{0, 1, 1};
+    const int nc = (pr.n + FC - 1) / FC;
     const int bh = pr.B * pr.H;
-    int P = kTargetCtas / bh;
-    P = P < 1 ? 1 : (P > pl.nc ? pl.nc : P);
-    if (P > kMaxSegments) P = kMaxSegments;
-    if ((long long)bh * P > kWsMaxFlags) P = 1;
-    pl.L = (pl.nc + P - 1) / P;
-    pl.P = (pl.nc + pl.L - 1) / pl.L;
-    return pl;
+    double tbest = 1e30;
+    const int pmax = nc < kMaxSegments ? nc : kMaxSegments;
+    for (int P = 1; P <= pmax; ++P) {
+        const int L = (nc + P - 1) / P;
+        if ((nc + L - 1) / L != P) continue;
+        if (P > 1 && (long long)bh * P > kWsMaxFlags) break;
+        const long long waves = ((long long)bh * P + kSMs - 1) / kSMs;
+        const double t = waves * L * (kMain + (P > 1 ? kPre : 0.0)) + (P - 1) * kFold + (P > 1 ? kFlag : 0.0);
+        if (t < tbest) {
+            tbest = t;
+            best = Plan{nc, P, L};
+        }
+    }
+    best.nc = nc;
+    return best;
 }
 
 struct WsLayout {
@@ -837,6 +887,35 @@ int launch_fused(const Problem &pr, void *ws, cudaStream_t st) {
     FusedParams p;
     memset(&p, 0, sizeof(p));
     char *w = static_cast<char *>(ws);
+    const CUtensorMapDataType dt16 =
+        pr.dtype == GTR_GLA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    const uint64_t bh = (uint64_t)pr.B * pr.H;
+    int boxh = FC;
+    if (pr.dir >= 2) {
+        boxh = 1;
+        while (boxh < FC && pr.gh % (2 * boxh) == 0) boxh *= 2;
+        if (boxh < 8) boxh = 0;
+    }
+    auto enc = [&](CUtensorMap *m, const void *base, CUtensorMapDataType dt, uint64_t es, bool sw) {
+        if (boxh == 0)  // [BH*n][64], one row per box (gathers)
+            return encode_rows_map(m, base, dt, (int)es, bh * pr.n, FD, sw);
+        if (pr.dir < 2) {  // [BH][n][64]
+            const uint64_t dims[3] = {FD, (uint64_t)pr.n, bh};
+            const uint64_t str[2] = {FD * es, (uint64_t)pr.n * FD * es};
+            const uint32_t box[3] = {FD, FC, 1};
+            return encode_tile_map(m, base, dt, 3, dims, str, box, sw);
+        }
+        // [BH][gh][gw][64]
+        const uint64_t dims[4] = {FD, (uint64_t)pr.gw, (uint64_t)pr.gh, bh};
+        const uint64_t str[3] = {FD * es, (uint64_t)pr.gw * FD * es, (uint64_t)pr.n * FD * es};
+        const uint32_t box[4] = {FD, 1, (uint32_t)boxh, 1};
+        return encode_tile_map(m, base, dt, 4, dims, str, box, sw);
+    };
+    if (enc(&p.tm_q, pr.q, dt16, 2, false) || enc(&p.tm_k, pr.k, dt16, 2, false) ||
+        enc(&p.tm_v, pr.v, dt16, 2, true) ||
+        enc(&p.tm_la, pr.la, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, false))
+        return GTR_GLA_ERR_CUDA;
+    p.boxh = boxh;
     p.q = pr.q;
     p.k = pr.k;
     p.v = pr.v;

@@ -38,6 +38,11 @@ int ensure_smem(const void *func, size_t bytes);
 int encode_rows_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int esize,
                     uint64_t rows, int cols, bool swizzle128);
 
+// Encode a tiled TMA map of rank 2..5 (tensormap.cu); 0 on success.
+int encode_tile_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int rank,
+                    const uint64_t *dims, const uint64_t *strides, const uint32_t *box,
+                    bool swizzle128);
+
 // Single-kernel tensor-core path (gla_fused.cu): fp16/bf16, d_k = d_v = 64, chunk 64.
 bool fused_supported(const Problem &p);
 size_t fused_workspace_bytes(const Problem &p);

@@ -41,4 +41,27 @@ int encode_rows_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, in
     return r == CUDA_SUCCESS ? 0 : 1;
 }
 
+// A tiled view of rank 2..5 (dims innermost first, strides in bytes for
+// dims 1..rank-1); loads of `box` elements start at any coordinate, elements
+// outside the tensor read as zero.
+int encode_tile_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int rank,
+                    const uint64_t *dims, const uint64_t *strides, const uint32_t *box,
+                    bool swizzle128) {
+    auto fn = encode_fn();
+    if (!fn || rank < 2 || rank > 5) return 1;
+    cuuint64_t d[5], st[4];
+    cuuint32_t b[5], e[5];
+    for (int i = 0; i < rank; ++i) {
+        d[i] = dims[i];
+        b[i] = box[i];
+        e[i] = 1;
+    }
+    for (int i = 0; i < rank - 1; ++i) st[i] = strides[i];
+    CUresult r = fn(m, dt, rank, const_cast<void *>(base), d, st, b, e,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? 0 : 1;
+}
+
 }  // namespace gtr
