@@ -68,15 +68,18 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kSpanLimit = 80.f;  // max -g (natural log) for the factorised scores
 
 // One pipeline stage (byte offsets from the stage base, every tile 1024-aligned).
-constexpr uint32_t ST_Q = 0;       // q  [64 tok][128 B] plain rows; later K~ (tf32, 16 KB, with ST_K)
-constexpr uint32_t ST_K = 8192;    // k  [64 tok][128 B] plain rows
-constexpr uint32_t ST_V = 16384;   // v  [64 tok][128 B] SW128 (MN-major MMA operand)
-constexpr uint32_t ST_LA = 24576;  // log_alpha [64 tok][256 B] fp32; later Q^ (tf32, 16 KB)
-constexpr uint32_t ST_KH = 40960;  // K^ [64 i][128 B] SW128 K-major
-constexpr uint32_t ST_BYTES = 49152;
-constexpr uint32_t ST_KT = ST_Q, ST_QH = ST_LA;
-constexpr uint32_t OFF_SB = kStages * ST_BYTES;  // S^T tf32 K-major [2][16 KB]
-constexpr uint32_t OFF_A = OFF_SB + 2 * 16384;   // A f16/bf16 K-major [2][8 KB]
+// Bytes [0, 32K) are the B operand of the merged product [scores | q S]: a
+// tf32 K-major tile [2 blocks of 32 K][128 rows][128 B], rows 0-63 K~
+// (tokens, written over q and k) and rows 64-127 S^T (value dims: the state
+// entering this chunk, written by the epilogue warps).
+constexpr uint32_t ST_Q = 0;       // q  [64 tok][128 B] plain rows -> K~, first 32 K
+constexpr uint32_t ST_K = 16384;   // k  [64 tok][128 B] plain rows -> K~, second 32 K
+constexpr uint32_t ST_LA = 32768;  // log_alpha [64 tok][256 B] fp32 -> Q^ (tf32, 16 KB)
+constexpr uint32_t ST_V = 49152;   // v  [64 tok][128 B] SW128 (MN-major MMA operand)
+constexpr uint32_t ST_KH = 57344;  // K^ [64 i][128 B] SW128 K-major
+constexpr uint32_t ST_BYTES = 65536;
+constexpr uint32_t ST_B1 = 0, ST_QH = ST_LA;
+constexpr uint32_t OFF_A = kStages * ST_BYTES;  // A f16/bf16 K-major [2][8 KB]
 constexpr uint32_t OFF_MISC = OFF_A + 2 * 8192;
 constexpr uint32_t MISC_ROWS = 0;     // int   [kStages][64] global row of each token
 constexpr uint32_t MISC_GAM = 768;    // float [kStages][64] e^{g}
@@ -88,9 +91,11 @@ constexpr uint32_t SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment sl
 static_assert(SMEM_BYTES <= 232448, "shared memory");
 
 constexpr uint32_t kTmemCols = 512;
-// TMEM columns (M = 64 results, lanes 32 q + 0..15): scores, dS^T, o (two
-// buffers each, by chunk parity) and the pre-pass aggregate.
-constexpr uint32_t TM_SC = 0, TM_DS = 128, TM_O = 256, TM_PRE = 384;
+// TMEM columns (M = 64 results, lanes 32 q + 0..15): three regions of 128
+// columns, [scores | o] of chunk k in region k % 3; dS^T in two buffers by
+// chunk parity; the pre-pass aggregate borrows region 2 (free until main
+// chunk 2, which is issued only after the aggregate has been published).
+constexpr uint32_t TM_R = 0, TM_DS = 384, TM_PRE = 256;
 
 struct FusedParams {
     // Tiled views of q, k, v, log_alpha.  Row scans (L->R, R->L): [BH][n][64],
@@ -202,6 +207,11 @@ __device__ __forceinline__ uint32_t tf32_kmaj(int row, int k) {
     return (k >> 5) * 8192 + sw128(row, (k & 31) >> 2) + (k & 3) * 4;
 }
 
+// the same for the stage's 128-row B tile (rows 0-63 K~, 64-127 S^T)
+__device__ __forceinline__ uint32_t b1_off(int row, int k) {
+    return (k >> 5) * 16384 + sw128(row, (k & 31) >> 2) + (k & 3) * 4;
+}
+
 // A shared-memory descriptor advanced by `bytes` (the start address field
 // holds addr >> 4 in its low 14 bits; smem addresses stay far below 256 KiB).
 __device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) {
@@ -228,8 +238,8 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
     int *sFlag = reinterpret_cast<int *>(sm + OFF_MISC + MISC_FLAG);
 
     __shared__ uint64_t bar_full[kStages], bar_empty[kStages], bar_op[kStages];
-    __shared__ uint64_t bar_sc[2], bar_o[2], bar_a[2], bar_s[2];
-    __shared__ uint64_t bar_pre, bar_owpre, bar_fin;
+    __shared__ uint64_t bar_sc[2], bar_o[2], bar_a[2], bar_s[2], bar_ds[2];
+    __shared__ uint64_t bar_pre, bar_owpre, bar_fin, bar_pub;
     __shared__ uint32_t s_tmem;
     __shared__ int s_ticket, s_last;
     __shared__ volatile int s_abort;
@@ -245,12 +255,14 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
         for (int b = 0; b < 2; ++b) {
             mbar_init(&bar_sc[b], 1);
             mbar_init(&bar_o[b], 1);
+            mbar_init(&bar_ds[b], 1);
             mbar_init(&bar_a[b], kEpiThreads);
             mbar_init(&bar_s[b], kEpiThreads);
         }
         mbar_init(&bar_pre, 1);
         mbar_init(&bar_owpre, kOpThreads);
         mbar_init(&bar_fin, 1);
+        mbar_init(&bar_pub, kEpiThreads);
         fence_mbar_init();
         s_ticket = (int)atomicAdd(&p.ctr[0], 1u);
         s_abort = 0;
@@ -368,69 +380,85 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
     } else if (warp == kWarpMma) {
         // ---------------------------------------------------------- MMA issue
         if (lane == 0) {
-            const uint32_t id_tf = idesc(2, 64, 64, 0, 0);     // tf32, both K-major
+            const uint32_t id_tf = idesc(2, 64, 128, 0, 0);    // tf32, both K-major, N = 128
+            const uint32_t id_tf64 = idesc(2, 64, 64, 0, 0);   // the same, N = 64
             const uint32_t id_av = idesc(kFmt, 64, 64, 0, 1);  // A K-major, V as B (MN-major)
             const uint32_t id_vk = idesc(kFmt, 64, 64, 1, 0);  // V^T as A (MN-major), K^ as B
+            // descriptors of stage 0 / buffer 0; stage s adds s * ST_BYTES (the
+            // start field holds address >> 4, far from overflowing)
             const uint32_t sbase = smem_u32(sm);
-            auto dq = [&](uint32_t off) { return sdesc_sw128(sbase + off, 16, 1024); };
-            auto dv = [&](uint32_t off) { return sdesc_sw128(sbase + off, 8192, 1024); };
+            const uint64_t d_qh = sdesc_sw128(sbase + ST_QH, 16, 1024);
+            const uint64_t d_b1 = sdesc_sw128(sbase + ST_B1, 16, 1024);
+            const uint64_t d_v = sdesc_sw128(sbase + ST_V, 8192, 1024);
+            const uint64_t d_kh = sdesc_sw128(sbase + ST_KH, 16, 1024);
+            const uint64_t d_a = sdesc_sw128(sbase + OFF_A, 16, 1024);
+            auto st_desc = [](uint64_t d, int s) { return d + (uint64_t)(s * (ST_BYTES >> 4)); };
             for (int it = 0; it < npre; ++it) {  // pre-pass: A_seg^T += V^T K^
                 const int s = it % kStages;
                 pwait(&bar_op[s], (it / kStages) & 1, &s_abort, p.err);
                 tc_fence_after_sync();
                 fence_proxy_async_smem();
-                const uint32_t so = s * ST_BYTES;
+                const uint64_t dv = st_desc(d_v, s), dk = st_desc(d_kh, s);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_f16(tbase + TM_PRE, desc_add(dv(so + ST_V), ks * 2048),
-                            desc_add(dq(so + ST_KH), ks * 32), id_vk, (it > 0 || ks > 0) ? 1u : 0u);
+                    mma_f16(tbase + TM_PRE, desc_add(dv, ks * 2048), desc_add(dk, ks * 32), id_vk,
+                            (it > 0 || ks > 0) ? 1u : 0u);
                 mma_commit(&bar_empty[s]);
             }
             if (npre > 0) mma_commit(&bar_pre);
-            // chunk k: scores and dS^T (needs its operands)
-            auto issue_sc = [&](int k) {
+            // o(k) += A_k V_k, then release chunk k's stage
+            auto issue_av = [&](int k) {
+                const int s = (npre + k) % kStages;
+                pwait(&bar_a[k & 1], (k >> 1) & 1, &s_abort, p.err);
+                tc_fence_after_sync();
+                fence_proxy_async_smem();
+                const uint64_t dv = st_desc(d_v, s), da = d_a + (uint64_t)((k & 1) * (8192 >> 4));
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_f16(tbase + TM_R + 128 * (k % 3) + 64, desc_add(da, ks * 32), desc_add(dv, ks * 2048),
+                            id_av, 1u);
+                mma_commit(&bar_o[k & 1]);
+                mma_commit(&bar_empty[s]);
+            };
+            for (int k = 0; k < L; ++k) {
                 const int it = npre + k, s = it % kStages;
+                // dS^T(k) = V^T K^ as soon as the operands are ready (the
+                // epilogue's state recursion only needs these)
                 pwait(&bar_op[s], (it / kStages) & 1, &s_abort, p.err);
                 tc_fence_after_sync();
                 fence_proxy_async_smem();
-                const uint32_t so = s * ST_BYTES, b = k & 1;
-                if (!sFlag[s]) {
+                {
+                    const uint64_t dv = st_desc(d_v, s), dk = st_desc(d_kh, s);
 #pragma unroll
-                    for (int ks = 0; ks < 8; ++ks) {
-                        const uint32_t o = (ks >> 2) * 8192 + (ks & 3) * 32;
-                        mma_tf32(tbase + TM_SC + 64 * b, desc_add(dq(so + ST_QH), o),
-                                 desc_add(dq(so + ST_KT), o), id_tf, ks > 0 ? 1u : 0u);
-                    }
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_f16(tbase + TM_DS + 64 * (k & 1), desc_add(dv, ks * 2048), desc_add(dk, ks * 32),
+                                id_vk, ks > 0 ? 1u : 0u);
+                    mma_commit(&bar_ds[k & 1]);
                 }
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_f16(tbase + TM_DS + 64 * b, desc_add(dv(so + ST_V), ks * 2048),
-                            desc_add(dq(so + ST_KH), ks * 32), id_vk, ks > 0 ? 1u : 0u);
-                mma_commit(&bar_sc[b]);
-            };
-            if (L > 0) issue_sc(0);
-            for (int k = 0; k < L; ++k) {
-                const int it = npre + k, s = it % kStages;
-                const uint32_t so = s * ST_BYTES, b = k & 1;
-                // state k (input of chunk k) is in SB[b]; chunk k-1's dS^T has been consumed
-                pwait(&bar_s[b], (k >> 1) & 1, &s_abort, p.err);
-                if (k + 1 < L) issue_sc(k + 1);
-                pwait(&bar_a[b], (k >> 1) & 1, &s_abort, p.err);
+                // [scores | o] = Q^ [K~ ; S_k^T]^T once state k is in the stage
+                pwait(&bar_s[k & 1], (k >> 1) & 1, &s_abort, p.err);
                 tc_fence_after_sync();
                 fence_proxy_async_smem();
+                {
+                    const uint64_t dq = st_desc(d_qh, s), db = st_desc(d_b1, s);
+                    if (!sFlag[s]) {
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {  // o = Q^ S_in
-                    const uint32_t o = (ks >> 2) * 8192 + (ks & 3) * 32;
-                    mma_tf32(tbase + TM_O + 64 * b, desc_add(dq(so + ST_QH), o),
-                             desc_add(dq(OFF_SB + 16384 * b), o), id_tf, ks > 0 ? 1u : 0u);
+                        for (int ks = 0; ks < 8; ++ks)
+                            mma_tf32(tbase + TM_R + 128 * (k % 3), desc_add(dq, (ks >> 2) * 8192 + (ks & 3) * 32),
+                                     desc_add(db, (ks >> 2) * 16384 + (ks & 3) * 32), id_tf, ks > 0 ? 1u : 0u);
+                    } else {  // exact scores are already in TMEM: only o = Q^ S (B rows 64-127)
+#pragma unroll
+                        for (int ks = 0; ks < 8; ++ks)
+                            mma_tf32(tbase + TM_R + 128 * (k % 3) + 64,
+                                     desc_add(dq, (ks >> 2) * 8192 + (ks & 3) * 32),
+                                     desc_add(db, (ks >> 2) * 16384 + 8192 + (ks & 3) * 32), id_tf64,
+                                     ks > 0 ? 1u : 0u);
+                    }
+                    mma_commit(&bar_sc[k & 1]);
                 }
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)  // o += A V
-                    mma_f16(tbase + TM_O + 64 * b, desc_add(dq(OFF_A + 8192 * b), ks * 32),
-                            desc_add(dv(so + ST_V), ks * 2048), id_av, 1u);
-                mma_commit(&bar_o[b]);
-                mma_commit(&bar_empty[s]);
+                if (k > 0) issue_av(k - 1);
             }
+            if (L > 0) issue_av(L - 1);
             mma_commit(&bar_fin);
             pwait(&bar_fin, 0, &s_abort, p.err);
         }
@@ -553,7 +581,10 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
                         st2(lat + pr * 64 + p2, make_float2(cb.x * kLog2e, cb.y * kLog2e));
                     }
                     named_bar_sync(kBarOp, kOpThreads);
-                    if (k >= 2) gwait(opl, kBarOp, kOpThreads, &bar_a[k & 1], ((k >> 1) - 1) & 1, &s_abort, p.err);
+                    // TMEM region k % 3 is free: its last chunk (k - 3) was masked
+                    // before this stage could be refilled; only region 2 during the
+                    // pre-pass's publication needs a wait
+                    if (k == 2 && npre > 0) gwait(opl, kBarOp, kOpThreads, &bar_pub, 0, &s_abort, p.err);
                     const int qd = warp & 3, r0 = 16 * qd + (lane >> 2), cq = 2 * (lane & 3);
                     uint32_t sc[32];
 #pragma unroll 1
@@ -570,7 +601,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
                         }
                         sc[e] = __float_as_uint(acc);
                     }
-                    tmem_st16x256(tbase + TM_SC + 64 * (k & 1) + ((uint32_t)(32 * qd) << 16), sc);
+                    tmem_st16x256(tbase + TM_R + 128 * (k % 3) + ((uint32_t)(32 * qd) << 16), sc);
                     tmem_st_wait();
                     named_bar_sync(kBarOp, kOpThreads);  // b is no longer read: Q^ may overwrite it
                 }
@@ -587,7 +618,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
                 // K^ = k . e^{g - b_u} (product of the alphas after u), K~ = K^ . e^{-g}
                 float2 f = ex2_2(after);
                 const float2 m = unsafe ? make_float2(0.f, 0.f) : ex2_2(make_float2(-g.x, -g.y));
-                uint8_t *kt = st + ST_KT;
+                uint8_t *kt = st + ST_B1;
                 float kh0[16], kh1[16];
 #pragma unroll
                 for (int kk = 15; kk >= 0; --kk) {
@@ -596,7 +627,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
                     kh0[kk] = h.x;
                     kh1[kk] = h.y;
                     const float2 t2 = fmul2(h, m);
-                    *reinterpret_cast<uint2 *>(kt + tf32_kmaj(u, p2)) = make_uint2(tf32_rn(t2.x), tf32_rn(t2.y));
+                    *reinterpret_cast<uint2 *>(kt + b1_off(u, p2)) = make_uint2(tf32_rn(t2.x), tf32_rn(t2.y));
                     f = fmul2(f, a[kk]);
                 }
                 store_kh(st + ST_KH, kh0, kh1);
@@ -628,6 +659,8 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
             uint32_t r[32];
             tmem_ld16x256(tbase + TM_PRE + lo, r);
             tmem_ld_wait();
+            tc_fence_before_sync();
+            mbar_arrive(&bar_pub);  // TMEM region 2 is free for the main pass
             float *dst = p.agg + slot * 4096;
 #pragma unroll
             for (int x = 0; x < 32; x += 2) {
@@ -690,17 +723,18 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
                 for (int c = 0; c < 8; ++c) gt[c] = gtn[c];
             }
         }
-        // state 0 (the incoming state) -> SB[0]
-        auto store_state = [&](int b) {
-            uint8_t *sb = sm + OFF_SB + 16384 * b;
+        // state k^T (tf32) -> rows 64-127 of the B tile of the stage holding chunk k
+        auto store_state = [&](int stage) {
+            uint8_t *sb = sm + stage * ST_BYTES + ST_B1;
 #pragma unroll
             for (int x = 0; x < 32; x += 2) {
                 const int j = r0 + 8 * ((x >> 1) & 1), i = 8 * (x >> 2) + cq;
-                *reinterpret_cast<uint2 *>(sb + tf32_kmaj(j, i)) = make_uint2(tf32_rn(S[x]), tf32_rn(S[x + 1]));
+                *reinterpret_cast<uint2 *>(sb + b1_off(64 + j, i)) = make_uint2(tf32_rn(S[x]), tf32_rn(S[x + 1]));
             }
             fence_proxy_async_smem();
         };
-        store_state(0);
+        if (L > 0) store_state(npre % kStages);  // state 0: the incoming state
+        tc_fence_before_sync();
         mbar_arrive(&bar_s[0]);
 
         // output of chunk kp (its o is complete once bar_o says so)
@@ -710,7 +744,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
             ok = gwait(epl, kBarEpi, kEpiThreads, &bar_o[b], (kp >> 1) & 1, &s_abort, p.err) && ok;
             tc_fence_after_sync();
             uint32_t r[32];
-            tmem_ld16x256(tbase + TM_O + 64 * b + lo, r);
+            tmem_ld16x256(tbase + TM_R + 128 * (kp % 3) + 64 + lo, r);
             tmem_ld_wait();
             if (ok) {
 #pragma unroll
@@ -733,8 +767,6 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
             // the operand warps' release of this stage makes its row table,
             // length and gate factors visible here
             ok = gwait(epl, kBarEpi, kEpiThreads, &bar_op[s], (it / kStages) & 1, &s_abort, p.err) && ok;
-            ok = gwait(epl, kBarEpi, kEpiThreads, &bar_sc[b], (k >> 1) & 1, &s_abort, p.err) && ok;
-            tc_fence_after_sync();
             // stage-local values, read before the stage can be recycled
             const int *rows = sRows + s * 64;
             const int len = sLen[s];
@@ -742,10 +774,33 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
             float2 gam[8];
 #pragma unroll
             for (int c = 0; c < 8; ++c) gam[c] = ld2(sGam + s * 64 + 8 * c + cq);
-            // causal mask of the scores -> A[b] (rows t, K = s)
+            // 1. state update S_{k+1} = diag(e^{g}) S_k + dS_k  (S^T: scale column i),
+            //    written into the next chunk's stage (its previous chunk's
+            //    product, which read that spot, completed before bar_sc of
+            //    chunk k-2 was seen)
+            ok = gwait(epl, kBarEpi, kEpiThreads, &bar_ds[b], (k >> 1) & 1, &s_abort, p.err) && ok;
+            tc_fence_after_sync();
             {
                 uint32_t r[32];
-                tmem_ld16x256(tbase + TM_SC + 64 * b + lo, r);
+                tmem_ld16x256(tbase + TM_DS + 64 * b + lo, r);
+                tmem_ld_wait();
+#pragma unroll
+                for (int x = 0; x < 32; x += 2) {
+                    const float2 t = ffma2(gam[x >> 2], make_float2(S[x], S[x + 1]),
+                                           make_float2(__uint_as_float(r[x]), __uint_as_float(r[x + 1])));
+                    S[x] = t.x;
+                    S[x + 1] = t.y;
+                }
+            }
+            if (k + 1 < L) store_state((it + 1) % kStages);
+            tc_fence_before_sync();
+            mbar_arrive(&bar_s[(k + 1) & 1]);
+            // 2. causal mask of the scores -> A[b] (rows t, K = s)
+            ok = gwait(epl, kBarEpi, kEpiThreads, &bar_sc[b], (k >> 1) & 1, &s_abort, p.err) && ok;
+            tc_fence_after_sync();
+            {
+                uint32_t r[32];
+                tmem_ld16x256(tbase + TM_R + 128 * (k % 3) + lo, r);
                 tmem_ld_wait();
                 uint8_t *sa = sAbuf + 8192 * b;
                 // columns follow V's stage rows: token s at column s, or 63 - s
@@ -764,26 +819,11 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
             fence_proxy_async_smem();
             tc_fence_before_sync();
             mbar_arrive(&bar_a[b]);
-            if (k > 0) emit(k - 1);  // chunk k-1's product is done: SB[(k+1)&1] is free again
+            // 3. output of the previous chunk
+            if (k > 0) emit(k - 1);
             prow[0] = row0;
             prow[1] = row1;
             plen = len;
-            // state update S_{k+1} = diag(e^{g}) S_k + dS_k  (S^T: scale column i)
-            {
-                uint32_t r[32];
-                tmem_ld16x256(tbase + TM_DS + 64 * b + lo, r);
-                tmem_ld_wait();
-#pragma unroll
-                for (int x = 0; x < 32; x += 2) {
-                    const float2 t = ffma2(gam[x >> 2], make_float2(S[x], S[x + 1]),
-                                           make_float2(__uint_as_float(r[x]), __uint_as_float(r[x + 1])));
-                    S[x] = t.x;
-                    S[x + 1] = t.y;
-                }
-            }
-            if (k + 1 < L) store_state((k + 1) & 1);
-            tc_fence_before_sync();
-            mbar_arrive(&bar_s[(k + 1) & 1]);
         }
         if (L > 0) emit(L - 1);
         if (seg == p.P - 1 && p.final_state && ok) {
