@@ -59,9 +59,10 @@ namespace {
 constexpr int FC = 64;  // tokens per chunk
 constexpr int FD = 64;  // d_k = d_v
 constexpr int kStages = 3;
-constexpr int kThreads = 320;
-constexpr int kWarpLoad = 0, kWarpMma = 1, kWarpOp0 = 2, kWarpEpi0 = 6;
-constexpr int kOpThreads = 128, kEpiThreads = 128;
+constexpr int kOpWarps = 8, kEpiWarps = 8;
+constexpr int kWarpLoad = 0, kWarpMma = 1, kWarpOp0 = 2, kWarpEpi0 = kWarpOp0 + kOpWarps;
+constexpr int kThreads = 32 * (kWarpEpi0 + kEpiWarps);
+constexpr int kOpThreads = 32 * kOpWarps, kEpiThreads = 32 * kEpiWarps;
 constexpr int kBarOp = 1, kBarEpi = 2;  // named barrier ids
 constexpr int kMaxSegments = 64;        // segments per (b,h): bounds the fold
 constexpr float kLog2e = 1.4426950408889634f;
@@ -83,12 +84,14 @@ constexpr uint32_t OFF_A = kStages * ST_BYTES;  // A f16/bf16 K-major [2][8 KB]
 constexpr uint32_t OFF_MISC = OFF_A + 2 * 8192;
 constexpr uint32_t MISC_ROWS = 0;     // int   [kStages][64] global row of each token
 constexpr uint32_t MISC_GAM = 768;    // float [kStages][64] e^{g}
-constexpr uint32_t MISC_TOT = 1536;   // float [2][4][64] operand warps' row-block log sums
-constexpr uint32_t MISC_LEN = 3584;   // int   [kStages] tokens in the chunk
-constexpr uint32_t MISC_FLAG = 3600;  // int   [kStages] exact-score chunk
-constexpr uint32_t MISC_BYTES = 4096;
+constexpr uint32_t MISC_LEN = 1536;   // int   [kStages] tokens in the chunk
+constexpr uint32_t MISC_FLAG = 1552;  // int   [kStages] exact-score chunk
+constexpr uint32_t MISC_TOT = 2048;   // float [2][kOpWarps][64] operand warps' row-block log sums
+constexpr uint32_t MISC_BYTES = 8192;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory");
+static_assert(MISC_TOT + 2 * kOpWarps * 64 * 4 <= MISC_BYTES, "misc area");
+static_assert(FC % kOpWarps == 0 && FC / kOpWarps == 8, "operand warps own 8 tokens each");
 
 constexpr uint32_t kTmemCols = 512;
 // TMEM columns (M = 64 results, lanes 32 q + 0..15): three regions of 128
@@ -422,6 +425,9 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
             };
             for (int k = 0; k < L; ++k) {
                 const int it = npre + k, s = it % kStages;
+                // the previous chunk's A V first: it releases that chunk's stage
+                // as soon as its mask is done
+                if (k > 0) issue_av(k - 1);
                 // dS^T(k) = V^T K^ as soon as the operands are ready (the
                 // epilogue's state recursion only needs these)
                 pwait(&bar_op[s], (it / kStages) & 1, &s_abort, p.err);
@@ -456,7 +462,6 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
                     }
                     mma_commit(&bar_sc[k & 1]);
                 }
-                if (k > 0) issue_av(k - 1);
             }
             if (L > 0) issue_av(L - 1);
             mma_commit(&bar_fin);
@@ -465,30 +470,29 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
         __syncwarp();
     } else if (warp < kWarpEpi0) {
         // ------------------------------------------------------ operand warps
-        const int ow = warp - kWarpOp0;  // tokens 16 ow .. 16 ow + 15
-        const int p2 = 2 * lane;         // key dims p2, p2 + 1
-        const bool rev = p.dir & 1;      // token u sits in stage row 63 - u
+        constexpr int RW = FC / kOpWarps;  // tokens per thread
+        const int ow = warp - kWarpOp0;    // tokens RW ow .. RW ow + RW - 1
+        const int p2 = 2 * lane;           // key dims p2, p2 + 1
+        const bool rev = p.dir & 1;        // token u sits in stage row 63 - u
         const bool opl = (warp == kWarpOp0 && lane == 0);  // the group's polling thread
-        const int row0 = rev ? 63 - 16 * ow : 16 * ow;   // stage row of token 16 ow
-        const int rstep = rev ? -1 : 1;                   // stage-row step per token
-        // K^ (the K index of V^T K^ follows V's stage rows): this thread's 16
-        // tokens occupy the 16-byte chunks kc0, kc0 + 1 of rows p2, p2 + 1
-        const int kc0 = rev ? 6 - 2 * ow : 2 * ow;
+        const int row0 = rev ? 63 - RW * ow : RW * ow;    // stage row of token RW ow
+        const int rstep = rev ? -1 : 1;                    // stage-row step per token
+        // K^ (the K index of V^T K^ follows V's stage rows): this thread's RW
+        // tokens fill the 16-byte chunk kc0 of rows p2, p2 + 1
+        const int kc0 = rev ? 7 - ow : ow;
         auto store_kh = [&](uint8_t *kh, float *kh0, float *kh1) {
             if (rev) {  // stage-row order is reversed token order
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
+                for (int j = 0; j < RW / 2; ++j) {
                     const float t0 = kh0[j], t1 = kh1[j];
-                    kh0[j] = kh0[15 - j];
-                    kh0[15 - j] = t0;
-                    kh1[j] = kh1[15 - j];
-                    kh1[15 - j] = t1;
+                    kh0[j] = kh0[RW - 1 - j];
+                    kh0[RW - 1 - j] = t0;
+                    kh1[j] = kh1[RW - 1 - j];
+                    kh1[RW - 1 - j] = t1;
                 }
             }
             *reinterpret_cast<uint4 *>(kh + sw128(p2, kc0)) = pack8<T>(kh0);
-            *reinterpret_cast<uint4 *>(kh + sw128(p2, kc0 + 1)) = pack8<T>(kh0 + 8);
             *reinterpret_cast<uint4 *>(kh + sw128(p2 + 1, kc0)) = pack8<T>(kh1);
-            *reinterpret_cast<uint4 *>(kh + sw128(p2 + 1, kc0 + 1)) = pack8<T>(kh1 + 8);
         };
         float2 gafter = make_float2(0.f, 0.f);
         for (int it = 0; it < n_items; ++it) {
@@ -499,27 +503,26 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
             uint8_t *st = sm + s * ST_BYTES;
             const int len = sLen[s];
             // 1. this thread's gates, q and k (everything is read before the
-            //    in-place overwrites below)
-            //    Loads are unconditional (every stage row is valid memory) and
-            //    tokens past the end are zeroed afterwards: no branch between
-            //    the loads, so they are all in flight at once.
-            float2 a[16];
-            uint32_t qw[16], kw[16];
+            //    in-place overwrites below).  Loads are unconditional (every
+            //    stage row is valid memory) and tokens past the end are zeroed
+            //    afterwards: no branch between the loads, all in flight at once.
+            float2 a[RW];
+            uint32_t qw[RW], kw[RW];
             float2 l = make_float2(0.f, 0.f);
-            const int nin = len - 16 * ow;  // this thread's tokens kk < nin are real
+            const int nin = len - RW * ow;  // this thread's tokens kk < nin are real
             {
                 const float *lr = reinterpret_cast<const float *>(st + ST_LA) + row0 * 64 + p2;
                 const uint8_t *kr = st + ST_K + row0 * 128 + p2 * 2;
                 const uint8_t *qr = st + ST_Q + row0 * 128 + p2 * 2;
-                float2 x[16];
+                float2 x[RW];
 #pragma unroll
-                for (int kk = 0; kk < 16; ++kk) {
+                for (int kk = 0; kk < RW; ++kk) {
                     x[kk] = ld2(lr + kk * rstep * 64);
                     kw[kk] = *reinterpret_cast<const uint32_t *>(kr + kk * rstep * 128);
                     qw[kk] = *reinterpret_cast<const uint32_t *>(qr + kk * rstep * 128);
                 }
 #pragma unroll
-                for (int kk = 0; kk < 16; ++kk) {
+                for (int kk = 0; kk < RW; ++kk) {
                     const bool in = kk < nin;
                     x[kk] = in ? x[kk] : make_float2(0.f, 0.f);
                     kw[kk] = in ? kw[kk] : 0u;
@@ -529,13 +532,13 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
                     a[kk] = ex2_2(x[kk]);
                 }
             }
-            float *tot = sTot + (it & 1) * 256;
+            float *tot = sTot + (it & 1) * (kOpWarps * 64);
             st2(tot + ow * 64 + p2, l);
             named_bar_sync(kBarOp, kOpThreads);
             // 2. where this thread's rows sit in the chunk
             float2 before = make_float2(0.f, 0.f), g = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int o = 0; o < 4; ++o) {
+            for (int o = 0; o < kOpWarps; ++o) {
                 const float2 t = ld2(tot + o * 64 + p2);
                 if (o < ow) {
                     before.x += t.x;
@@ -548,11 +551,10 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
             if (pre) {
                 // K^ relative to the segment end: k . e^{G_after + (gates after u in the chunk)}
                 float2 f = ex2_2(make_float2(gafter.x + after.x, gafter.y + after.y));
-                float kh0[16], kh1[16];
+                float kh0[RW], kh1[RW];
 #pragma unroll
-                for (int kk = 15; kk >= 0; --kk) {
-                    const float2 kv = Pack2<T>::unpack(kw[kk]);
-                    const float2 h = fmul2(kv, f);
+                for (int kk = RW - 1; kk >= 0; --kk) {
+                    const float2 h = fmul2(Pack2<T>::unpack(kw[kk]), f);
                     kh0[kk] = h.x;
                     kh1[kk] = h.y;
                     f = fmul2(f, a[kk]);
@@ -573,8 +575,8 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
                     float2 cb = before;
                     float *lat = reinterpret_cast<float *>(st + ST_LA);
 #pragma unroll
-                    for (int kk = 0; kk < 16; ++kk) {
-                        const int u = 16 * ow + kk, pr = rev ? 63 - u : u;
+                    for (int kk = 0; kk < RW; ++kk) {
+                        const int u = RW * ow + kk, pr = rev ? 63 - u : u;
                         const float2 x = (u < len) ? ld2(lat + pr * 64 + p2) : make_float2(0.f, 0.f);
                         cb.x += x.x;
                         cb.y += x.y;
@@ -585,11 +587,14 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
                     // before this stage could be refilled; only region 2 during the
                     // pre-pass's publication needs a wait
                     if (k == 2 && npre > 0) gwait(opl, kBarOp, kOpThreads, &bar_pub, 0, &s_abort, p.err);
-                    const int qd = warp & 3, r0 = 16 * qd + (lane >> 2), cq = 2 * (lane & 3);
-                    uint32_t sc[32];
+                    // this warp's part of the M = 64 score tile: its lane quadrant,
+                    // one half of the columns
+                    const int qd = warp & 3, hc = (ow >> 2) * 32;
+                    const int r0 = 16 * qd + (lane >> 2), cq = 2 * (lane & 3);
+                    uint32_t sc[16];
 #pragma unroll 1
-                    for (int e = 0; e < 32; ++e) {
-                        const int t = r0 + 8 * ((e >> 1) & 1), sx = 8 * (e >> 2) + cq + (e & 1);
+                    for (int e = 0; e < 16; ++e) {
+                        const int t = r0 + 8 * ((e >> 1) & 1), sx = hc + 8 * (e >> 2) + cq + (e & 1);
                         float acc = 0.f;
                         if (sx <= t && t < len) {
                             const int pt = rev ? 63 - t : t, ps = rev ? 63 - sx : sx;
@@ -601,7 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
                         }
                         sc[e] = __float_as_uint(acc);
                     }
-                    tmem_st16x256(tbase + TM_R + 128 * (k % 3) + ((uint32_t)(32 * qd) << 16), sc);
+                    tmem_st16x256_x4(tbase + TM_R + 128 * (k % 3) + hc + ((uint32_t)(32 * qd) << 16), sc);
                     tmem_st_wait();
                     named_bar_sync(kBarOp, kOpThreads);  // b is no longer read: Q^ may overwrite it
                 }
@@ -609,8 +614,8 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
                 float2 e = ex2_2(before);
                 uint8_t *qh = st + ST_QH;
 #pragma unroll
-                for (int kk = 0; kk < 16; ++kk) {
-                    const int u = 16 * ow + kk;
+                for (int kk = 0; kk < RW; ++kk) {
+                    const int u = RW * ow + kk;
                     e = fmul2(e, a[kk]);
                     const float2 v = fmul2(Pack2<T>::unpack(qw[kk]), e);
                     *reinterpret_cast<uint2 *>(qh + tf32_kmaj(u, p2)) = make_uint2(tf32_rn(v.x), tf32_rn(v.y));
@@ -619,10 +624,10 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
                 float2 f = ex2_2(after);
                 const float2 m = unsafe ? make_float2(0.f, 0.f) : ex2_2(make_float2(-g.x, -g.y));
                 uint8_t *kt = st + ST_B1;
-                float kh0[16], kh1[16];
+                float kh0[RW], kh1[RW];
 #pragma unroll
-                for (int kk = 15; kk >= 0; --kk) {
-                    const int u = 16 * ow + kk;
+                for (int kk = RW - 1; kk >= 0; --kk) {
+                    const int u = RW * ow + kk;
                     const float2 h = fmul2(Pack2<T>::unpack(kw[kk]), f);
                     kh0[kk] = h.x;
                     kh1[kk] = h.y;
@@ -642,35 +647,40 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
         }
     } else {
         // ----------------------------------------------------- epilogue warps
-        const int qd = warp & 3;                       // TMEM lane quadrant
-        const uint32_t lo = (uint32_t)(32 * qd) << 16;
-        const int r0 = 16 * qd + (lane >> 2);          // rows r0 and r0 + 8
-        const int cq = 2 * (lane & 3);                 // columns 8 c + cq + {0, 1}
+        // Two warps per TMEM lane quadrant, one per half of the columns; a
+        // thread holds rows r0, r0 + 8 and columns hc + 8 c + cq + {0, 1}
+        // (c = 0..3) of every M = 64 result: element x <-> row r0 + 8 ((x >> 1) & 1),
+        // column hc + 8 (x >> 2) + cq + (x & 1).
+        const int qd = warp & 3;
+        const int hc = ((warp - kWarpEpi0) >> 2) * 32;
+        const uint32_t lo = ((uint32_t)(32 * qd) << 16) + hc;
+        const int r0 = 16 * qd + (lane >> 2);
+        const int cq = 2 * (lane & 3);
         const bool rev = p.dir & 1;
         const bool epl = (warp == kWarpEpi0 && lane == 0);  // the group's polling thread
         bool ok = true;
-        float S[32];  // S^T[j][i]: j = r0 + 8 ((x >> 1) & 1), i = 8 (x >> 2) + cq + (x & 1)
+        float S[16];  // S^T[j][i] of this thread's elements
 #pragma unroll
-        for (int x = 0; x < 32; ++x) S[x] = 0.f;
+        for (int x = 0; x < 16; ++x) S[x] = 0.f;
 
         if (npre > 0) {  // publish the aggregate A_seg^T and raise this segment's flag
             ok = gwait(epl, kBarEpi, kEpiThreads, &bar_pre, 0, &s_abort, p.err, 256) && ok;
             tc_fence_after_sync();
-            uint32_t r[32];
-            tmem_ld16x256(tbase + TM_PRE + lo, r);
+            uint32_t r[16];
+            tmem_ld16x256_x4(tbase + TM_PRE + lo, r);
             tmem_ld_wait();
             tc_fence_before_sync();
             mbar_arrive(&bar_pub);  // TMEM region 2 is free for the main pass
             float *dst = p.agg + slot * 4096;
 #pragma unroll
-            for (int x = 0; x < 32; x += 2) {
-                const int j = r0 + 8 * ((x >> 1) & 1), i = 8 * (x >> 2) + cq;
+            for (int x = 0; x < 16; x += 2) {
+                const int j = r0 + 8 * ((x >> 1) & 1), i = hc + 8 * (x >> 2) + cq;
                 st2(dst + j * 64 + i, make_float2(__uint_as_float(r[x]), __uint_as_float(r[x + 1])));
             }
             ok = gwait(epl, kBarEpi, kEpiThreads, &bar_owpre, 0, &s_abort, p.err) && ok;
             __threadfence();
             named_bar_sync(kBarEpi, kEpiThreads);
-            if (warp == kWarpEpi0 && lane == 0 && ok) st_release(p.flag + slot, 1);
+            if (epl && ok) st_release(p.flag + slot, 1);
         }
         if (seg > 0) {  // fold the earlier segments' aggregates, nearest first
             if (warp == kWarpEpi0) {
@@ -683,29 +693,29 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
             }
             named_bar_sync(kBarEpi, kEpiThreads);
             if (s_abort) ok = false;
-            float2 acc[8];  // log-gate sums of the segments between the source and this one
+            float2 acc[4];  // log-gate sums of the segments between the source and this one
 #pragma unroll
-            for (int c = 0; c < 8; ++c) acc[c] = make_float2(0.f, 0.f);
+            for (int c = 0; c < 4; ++c) acc[c] = make_float2(0.f, 0.f);
             // software-pipelined: the next aggregate's loads are in flight
             // while the current one is folded
-            float2 v[16], gt[8], vn[16], gtn[8];
+            float2 v[8], gt[4], vn[8], gtn[4];
             auto load = [&](int d, float2 *vv, float2 *gg) {
                 const size_t src = (size_t)bh * p.P + (seg - 1 - d);
                 const float *ag = p.agg + src * 4096;
 #pragma unroll
-                for (int x = 0; x < 32; x += 2) {
-                    const int j = r0 + 8 * ((x >> 1) & 1), i = 8 * (x >> 2) + cq;
+                for (int x = 0; x < 16; x += 2) {
+                    const int j = r0 + 8 * ((x >> 1) & 1), i = hc + 8 * (x >> 2) + cq;
                     vv[x >> 1] = __ldcg(reinterpret_cast<const float2 *>(ag + j * 64 + i));
                 }
 #pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    gg[c] = __ldcg(reinterpret_cast<const float2 *>(p.aggg + src * 64 + 8 * c + cq));
+                for (int c = 0; c < 4; ++c)
+                    gg[c] = __ldcg(reinterpret_cast<const float2 *>(p.aggg + src * 64 + hc + 8 * c + cq));
             };
             if (ok) load(0, v, gt);
             for (int d = 0; d < seg && ok; ++d) {
                 if (d + 1 < seg) load(d + 1, vn, gtn);
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
+                for (int c = 0; c < 4; ++c) {
                     const float2 sc = ex2_2(acc[c]);
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
@@ -718,17 +728,17 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
                     acc[c].y += gt[c].y;
                 }
 #pragma unroll
-                for (int x = 0; x < 16; ++x) v[x] = vn[x];
+                for (int x = 0; x < 8; ++x) v[x] = vn[x];
 #pragma unroll
-                for (int c = 0; c < 8; ++c) gt[c] = gtn[c];
+                for (int c = 0; c < 4; ++c) gt[c] = gtn[c];
             }
         }
         // state k^T (tf32) -> rows 64-127 of the B tile of the stage holding chunk k
         auto store_state = [&](int stage) {
             uint8_t *sb = sm + stage * ST_BYTES + ST_B1;
 #pragma unroll
-            for (int x = 0; x < 32; x += 2) {
-                const int j = r0 + 8 * ((x >> 1) & 1), i = 8 * (x >> 2) + cq;
+            for (int x = 0; x < 16; x += 2) {
+                const int j = r0 + 8 * ((x >> 1) & 1), i = hc + 8 * (x >> 2) + cq;
                 *reinterpret_cast<uint2 *>(sb + b1_off(64 + j, i)) = make_uint2(tf32_rn(S[x]), tf32_rn(S[x + 1]));
             }
             fence_proxy_async_smem();
@@ -740,20 +750,19 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
         // output of chunk kp (its o is complete once bar_o says so)
         int prow[2] = {0, 0}, plen = 0;
         auto emit = [&](int kp) {
-            const int b = kp & 1;
-            ok = gwait(epl, kBarEpi, kEpiThreads, &bar_o[b], (kp >> 1) & 1, &s_abort, p.err) && ok;
+            ok = gwait(epl, kBarEpi, kEpiThreads, &bar_o[kp & 1], (kp >> 1) & 1, &s_abort, p.err) && ok;
             tc_fence_after_sync();
-            uint32_t r[32];
-            tmem_ld16x256(tbase + TM_R + 128 * (kp % 3) + 64 + lo, r);
+            uint32_t r[16];
+            tmem_ld16x256_x4(tbase + TM_R + 128 * (kp % 3) + 64 + lo, r);
             tmem_ld_wait();
             if (ok) {
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     if (r0 + 8 * h < plen) {
                         uint32_t *dst = reinterpret_cast<uint32_t *>(reinterpret_cast<T *>(p.out) +
-                                                                     (size_t)prow[h] * FD + cq);
+                                                                     (size_t)prow[h] * FD + hc + cq);
 #pragma unroll
-                        for (int c = 0; c < 8; ++c)
+                        for (int c = 0; c < 4; ++c)
                             dst[4 * c] = Pack2<T>::pack(__uint_as_float(r[4 * c + 2 * h]),
                                                         __uint_as_float(r[4 * c + 2 * h + 1]));
                     }
@@ -771,9 +780,9 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
             const int *rows = sRows + s * 64;
             const int len = sLen[s];
             const int row0 = rows[r0], row1 = rows[r0 + 8];
-            float2 gam[8];
+            float2 gam[4];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) gam[c] = ld2(sGam + s * 64 + 8 * c + cq);
+            for (int c = 0; c < 4; ++c) gam[c] = ld2(sGam + s * 64 + hc + 8 * c + cq);
             // 1. state update S_{k+1} = diag(e^{g}) S_k + dS_k  (S^T: scale column i),
             //    written into the next chunk's stage (its previous chunk's
             //    product, which read that spot, completed before bar_sc of
@@ -781,11 +790,11 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
             ok = gwait(epl, kBarEpi, kEpiThreads, &bar_ds[b], (k >> 1) & 1, &s_abort, p.err) && ok;
             tc_fence_after_sync();
             {
-                uint32_t r[32];
-                tmem_ld16x256(tbase + TM_DS + 64 * b + lo, r);
+                uint32_t r[16];
+                tmem_ld16x256_x4(tbase + TM_DS + 64 * b + lo, r);
                 tmem_ld_wait();
 #pragma unroll
-                for (int x = 0; x < 32; x += 2) {
+                for (int x = 0; x < 16; x += 2) {
                     const float2 t = ffma2(gam[x >> 2], make_float2(S[x], S[x + 1]),
                                            make_float2(__uint_as_float(r[x]), __uint_as_float(r[x + 1])));
                     S[x] = t.x;
@@ -799,20 +808,20 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
             ok = gwait(epl, kBarEpi, kEpiThreads, &bar_sc[b], (k >> 1) & 1, &s_abort, p.err) && ok;
             tc_fence_after_sync();
             {
-                uint32_t r[32];
-                tmem_ld16x256(tbase + TM_R + 128 * (k % 3) + lo, r);
+                uint32_t r[16];
+                tmem_ld16x256_x4(tbase + TM_R + 128 * (k % 3) + lo, r);
                 tmem_ld_wait();
                 uint8_t *sa = sAbuf + 8192 * b;
                 // columns follow V's stage rows: token s at column s, or 63 - s
-                // for reversed scans
-                // (column 63 - s = 16-byte chunk 7 ^ c, element 6 ^ cq, the pair swapped)
+                // for reversed scans (16-byte chunk 7 ^ c, element 6 ^ cq, the
+                // pair swapped)
                 const int cx = rev ? 7 : 0, ex = rev ? 6 : 0;
 #pragma unroll
-                for (int x = 0; x < 32; x += 2) {
-                    const int t = r0 + 8 * ((x >> 1) & 1), sx = 8 * (x >> 2) + cq;
+                for (int x = 0; x < 16; x += 2) {
+                    const int t = r0 + 8 * ((x >> 1) & 1), c = (hc >> 3) + (x >> 2), sx = 8 * c + cq;
                     const float v0 = (sx <= t) ? __uint_as_float(r[x]) : 0.f;
                     const float v1 = (sx + 1 <= t) ? __uint_as_float(r[x + 1]) : 0.f;
-                    *reinterpret_cast<uint32_t *>(sa + sw128(t, (x >> 2) ^ cx) + (cq ^ ex) * 2) =
+                    *reinterpret_cast<uint32_t *>(sa + sw128(t, c ^ cx) + (cq ^ ex) * 2) =
                         rev ? Pack2<T>::pack(v1, v0) : Pack2<T>::pack(v0, v1);
                 }
             }
@@ -829,8 +838,8 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
         if (seg == p.P - 1 && p.final_state && ok) {
             float *fs = p.final_state + (size_t)bh * 4096;
 #pragma unroll
-            for (int x = 0; x < 32; ++x) {
-                const int j = r0 + 8 * ((x >> 1) & 1), i = 8 * (x >> 2) + cq + (x & 1);
+            for (int x = 0; x < 16; ++x) {
+                const int j = r0 + 8 * ((x >> 1) & 1), i = hc + 8 * (x >> 2) + cq + (x & 1);
                 fs[i * 64 + j] = S[x];
             }
         }
