@@ -55,6 +55,26 @@ def workload_bytes(shape, dtype: str) -> int:
             + shape.B * shape.H * shape.d_k * shape.d_v * 4)
 
 
+def profiled_traffic(workload: str):
+    """DRAM bytes of one launch of the fused kernel for `workload`, from the
+    committed ncu summary, if that summary was taken on the current kernel
+    source (its sha256 prefix matches); else None."""
+    import hashlib
+    import re
+
+    prof = os.path.join(ROOT, "profiles", "gla_fused_kernel.md")
+    src = os.path.join(ROOT, "recurrent_vision_backbone_chunkwise_b200", "csrc", "gla_fused.cu")
+    if not (os.path.exists(prof) and os.path.exists(src)):
+        return None
+    text = open(prof).read()
+    m = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]{16})", text)
+    with open(src, "rb") as f:
+        if not m or hashlib.sha256(f.read()).hexdigest()[:16] != m.group(1):
+            return None
+    m = re.search(r"traffic_bytes_per_launch\s+" + re.escape(workload) + r"\s+(\d+)", text)
+    return int(m.group(1)) if m else None
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -337,7 +357,7 @@ def main():
                                "median": 1e3 * statistics.median(call_ms),
                                "min": 1e3 * min(call_ms)},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": None,
+                     "frac": achieved / peak, "traffic": profiled_traffic(args.config),
                      "peak_source": f"{peak_kind} copy bandwidth",
                      "bytes_per_call": call_bytes,
                      "timed_unit": "one library call (all kernels of one direction)"},
