@@ -97,9 +97,10 @@ int gtr_gla_fwd(const void *q, const void *k, const void *v, const float *log_al
  * the workspace chosen by the caller.
  *   dtype:     GTR_GLA_F16, GTR_GLA_BF16 or GTR_GLA_F32.
  *   chunk:     tokens per chunk, 32 or 64.  The result does not depend on it
- *              beyond rounding.  F16/BF16 with d_k = d_v = 64 and chunk 64 run
- *              the fused tensor-core kernel; every other combination runs the
- *              three-phase CUDA-core path.
+ *              beyond rounding.  F16/BF16 with chunk 64 run the fused
+ *              tensor-core kernel (head sizes of 128 as 64-wide parts, one
+ *              launch each); every other combination runs the three-phase
+ *              CUDA-core path.
  *   workspace: device buffer of at least gtr_gla_workspace_size(...) bytes,
  *              256-byte aligned, zero-filled before its first use.  Every call
  *              leaves it ready for the next one.  Calls that share a workspace

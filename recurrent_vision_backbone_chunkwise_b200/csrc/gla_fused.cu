@@ -116,6 +116,13 @@ struct FusedParams {
     unsigned *ctr;  // [0] ticket, [1] finished CTAs
     int *err;
     int n, gh, gw, dir, nc, P, L, BH;
+    // Head sizes of 128 run as 64-wide sub-problems (every key row of the
+    // state evolves on its own and every value column too; the output is
+    // the sum over the key halves): `out` and `final_state` point at the
+    // sub-problem's corner, ldo is the output row stride in elements,
+    // acc_out adds to what is already in `out`, fs_bh / fs_ld are the final
+    // state's (b,h) and row strides.
+    int ldo, acc_out, fs_bh, fs_ld;
     int boxh;  // rows per box (64 for row scans); 0: four-row gathers (column
                // scans whose grid_h is not a multiple of 8, where a box of V
                // could not start on its 128-byte swizzle atom)
@@ -760,11 +767,20 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
                 for (int h = 0; h < 2; ++h) {
                     if (r0 + 8 * h < plen) {
                         uint32_t *dst = reinterpret_cast<uint32_t *>(reinterpret_cast<T *>(p.out) +
-                                                                     (size_t)prow[h] * FD + hc + cq);
+                                                                     (size_t)prow[h] * p.ldo + hc + cq);
+                        if (p.acc_out) {  // second key half: add to the first half's output
 #pragma unroll
-                        for (int c = 0; c < 4; ++c)
-                            dst[4 * c] = Pack2<T>::pack(__uint_as_float(r[4 * c + 2 * h]),
-                                                        __uint_as_float(r[4 * c + 2 * h + 1]));
+                            for (int c = 0; c < 4; ++c) {
+                                const float2 o = Pack2<T>::unpack(dst[4 * c]);
+                                dst[4 * c] = Pack2<T>::pack(o.x + __uint_as_float(r[4 * c + 2 * h]),
+                                                            o.y + __uint_as_float(r[4 * c + 2 * h + 1]));
+                            }
+                        } else {
+#pragma unroll
+                            for (int c = 0; c < 4; ++c)
+                                dst[4 * c] = Pack2<T>::pack(__uint_as_float(r[4 * c + 2 * h]),
+                                                            __uint_as_float(r[4 * c + 2 * h + 1]));
+                        }
                     }
                 }
             }
@@ -836,11 +852,11 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
         }
         if (L > 0) emit(L - 1);
         if (seg == p.P - 1 && p.final_state && ok) {
-            float *fs = p.final_state + (size_t)bh * 4096;
+            float *fs = p.final_state + (size_t)bh * p.fs_bh;
 #pragma unroll
             for (int x = 0; x < 16; ++x) {
                 const int j = r0 + 8 * ((x >> 1) & 1), i = hc + 8 * (x >> 2) + cq + (x & 1);
-                fs[i * 64 + j] = S[x];
+                fs[(size_t)i * p.fs_ld + j] = S[x];
             }
         }
     }
@@ -923,16 +939,16 @@ WsLayout ws_layout(const Problem &pr, const Plan &pl) {
 
 bool fused_supported(const Problem &pr) {
     if (pr.dtype != GTR_GLA_F16 && pr.dtype != GTR_GLA_BF16) return false;
-    if (pr.dk != 64 || pr.dv != 64 || pr.chunk != 64) return false;
+    if ((pr.dk != 64 && pr.dk != 128) || (pr.dv != 64 && pr.dv != 128) || pr.chunk != 64) return false;
     if ((long long)pr.B * pr.H * pr.n >= (1LL << 31)) return false;
     return true;
 }
 
 size_t fused_workspace_bytes(const Problem &pr) { return ws_layout(pr, make_plan(pr)).total; }
 
-int launch_fused(const Problem &pr, void *ws, cudaStream_t st) {
-    const Plan pl = make_plan(pr);
-    const WsLayout wl = ws_layout(pr, pl);
+// One launch for the 64-wide sub-problem (key half kh, value half vh).
+static int launch_fused_part(const Problem &pr, const Plan &pl, const WsLayout &wl, void *ws,
+                             int kh, int vh, cudaStream_t st) {
     FusedParams p;
     memset(&p, 0, sizeof(p));
     char *w = static_cast<char *>(ws);
@@ -945,32 +961,44 @@ int launch_fused(const Problem &pr, void *ws, cudaStream_t st) {
         while (boxh < FC && pr.gh % (2 * boxh) == 0) boxh *= 2;
         if (boxh < 8) boxh = 0;
     }
-    auto enc = [&](CUtensorMap *m, const void *base, CUtensorMapDataType dt, uint64_t es, bool sw) {
-        if (boxh == 0)  // [BH*n][64], one row per box (gathers)
-            return encode_rows_map(m, base, dt, (int)es, bh * pr.n, FD, sw);
+    // views of the 64 columns starting at col0 of a [BH][n][ld] tensor
+    auto enc = [&](CUtensorMap *m, const void *base0, int ld, int col0, CUtensorMapDataType dt, uint64_t es,
+                   bool sw) {
+        const void *base = static_cast<const char *>(base0) + (size_t)col0 * es;
+        const uint64_t row = (uint64_t)ld * es;
+        if (boxh == 0) {  // [BH*n][64], one row per box (gathers)
+            const uint64_t dims[2] = {FD, bh * pr.n};
+            const uint64_t str[1] = {row};
+            const uint32_t box[2] = {FD, 1};
+            return encode_tile_map(m, base, dt, 2, dims, str, box, sw);
+        }
         if (pr.dir < 2) {  // [BH][n][64]
             const uint64_t dims[3] = {FD, (uint64_t)pr.n, bh};
-            const uint64_t str[2] = {FD * es, (uint64_t)pr.n * FD * es};
+            const uint64_t str[2] = {row, (uint64_t)pr.n * row};
             const uint32_t box[3] = {FD, FC, 1};
             return encode_tile_map(m, base, dt, 3, dims, str, box, sw);
         }
         // [BH][gh][gw][64]
         const uint64_t dims[4] = {FD, (uint64_t)pr.gw, (uint64_t)pr.gh, bh};
-        const uint64_t str[3] = {FD * es, (uint64_t)pr.gw * FD * es, (uint64_t)pr.n * FD * es};
+        const uint64_t str[3] = {row, (uint64_t)pr.gw * row, (uint64_t)pr.n * row};
         const uint32_t box[4] = {FD, 1, (uint32_t)boxh, 1};
         return encode_tile_map(m, base, dt, 4, dims, str, box, sw);
     };
-    if (enc(&p.tm_q, pr.q, dt16, 2, false) || enc(&p.tm_k, pr.k, dt16, 2, false) ||
-        enc(&p.tm_v, pr.v, dt16, 2, true) ||
-        enc(&p.tm_la, pr.la, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, false))
+    if (enc(&p.tm_q, pr.q, pr.dk, FD * kh, dt16, 2, false) || enc(&p.tm_k, pr.k, pr.dk, FD * kh, dt16, 2, false) ||
+        enc(&p.tm_v, pr.v, pr.dv, FD * vh, dt16, 2, true) ||
+        enc(&p.tm_la, pr.la, pr.dk, FD * kh, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, false))
         return GTR_GLA_ERR_CUDA;
     p.boxh = boxh;
     p.q = pr.q;
     p.k = pr.k;
     p.v = pr.v;
     p.la = pr.la;
-    p.out = pr.out;
-    p.final_state = pr.final_state;
+    p.out = static_cast<char *>(pr.out) + (size_t)FD * vh * 2;
+    p.ldo = pr.dv;
+    p.acc_out = kh > 0;
+    p.final_state = pr.final_state ? pr.final_state + (size_t)FD * kh * pr.dv + FD * vh : nullptr;
+    p.fs_bh = pr.dk * pr.dv;
+    p.fs_ld = pr.dv;
     p.agg = reinterpret_cast<float *>(w + wl.agg);
     p.aggg = reinterpret_cast<float *>(w + wl.aggg);
     p.flag = reinterpret_cast<int *>(w + wl.flag);
@@ -994,6 +1022,21 @@ int launch_fused(const Problem &pr, void *ws, cudaStream_t st) {
     }
     note_launch();
     return cudaPeekAtLastError() == cudaSuccess ? GTR_GLA_OK : GTR_GLA_ERR_CUDA;
+}
+
+// Head sizes of 128 run as 64-wide sub-problems, one launch each, in stream
+// order: first every value half of key half 0 (which writes the output),
+// then key half 1 (which adds to it).  The launches share the workspace; each
+// leaves its header zeroed for the next.
+int launch_fused(const Problem &pr, void *ws, cudaStream_t st) {
+    const Plan pl = make_plan(pr);
+    const WsLayout wl = ws_layout(pr, pl);
+    for (int kh = 0; kh < pr.dk / FD; ++kh)
+        for (int vh = 0; vh < pr.dv / FD; ++vh) {
+            const int rc = launch_fused_part(pr, pl, wl, ws, kh, vh, st);
+            if (rc != GTR_GLA_OK) return rc;
+        }
+    return GTR_GLA_OK;
 }
 
 }  // namespace gtr

@@ -72,7 +72,7 @@ extern "C" int gtr_gla_fwd_noalloc(const void *q, const void *k, const void *v,
     p.err = nullptr;
     int rc = check_problem(p);
     if (rc) return rc;
-    if (!fused_supported(p)) return GTR_GLA_ERR_HEAD_DIM;
+    if (!fused_supported(p) || p.dk != 64 || p.dv != 64) return GTR_GLA_ERR_HEAD_DIM;
     if (fused_workspace_bytes(p) > kNoAllocScratchBytes) return GTR_GLA_ERR_WORKSPACE;
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices)
