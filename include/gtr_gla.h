@@ -69,7 +69,7 @@ enum {
     GTR_GLA_ERR_DIRECTION = -4,   /* direction not in [0, 3]                      */
     GTR_GLA_ERR_ALIGN = -5,       /* a pointer is not 16-byte aligned             */
     GTR_GLA_ERR_DTYPE = -6,       /* dtype not one of GTR_GLA_F16/BF16/F32        */
-    GTR_GLA_ERR_CHUNK = -7,       /* chunk length not supported for this dtype    */
+    GTR_GLA_ERR_CHUNK = -7,       /* chunk length not supported for these sizes   */
     GTR_GLA_ERR_WORKSPACE = -8,   /* workspace NULL or smaller than required      */
     GTR_GLA_ERR_CUDA = -9,        /* a CUDA runtime call or launch failed         */
     GTR_GLA_ERR_TIMEOUT = -10,    /* a device-side wait gave up (gtr_gla_status)  */
@@ -96,7 +96,8 @@ int gtr_gla_fwd(const void *q, const void *k, const void *v, const float *log_al
  * gtr_gla_fwd_ex -- as gtr_gla_fwd with the I/O dtype, the chunk length and
  * the workspace chosen by the caller.
  *   dtype:     GTR_GLA_F16, GTR_GLA_BF16 or GTR_GLA_F32.
- *   chunk:     tokens per chunk, 32 or 64.  The result does not depend on it
+ *   chunk:     tokens per chunk: 32 or 64, or 128 when d_k = 64 (else
+ *              GTR_GLA_ERR_CHUNK).  The result does not depend on it
  *              beyond rounding.  F16/BF16 with chunk 64 run the fused
  *              tensor-core kernel (head sizes of 128 as 64-wide parts, one
  *              launch each); every other combination runs the three-phase

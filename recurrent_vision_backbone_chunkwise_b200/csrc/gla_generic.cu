@@ -304,6 +304,10 @@ template <typename T>
 static int launch_generic_chunk(const Problem &p, void *ws, cudaStream_t st) {
     if (p.chunk == 32) return launch_generic_dims<T, 32>(p, ws, st);
     if (p.chunk == 64) return launch_generic_dims<T, 64>(p, ws, st);
+    if (p.chunk == 128 && p.dk == 64) {  // d_k = 128 would not fit shared memory
+        if (p.dv == 64) return launch_generic_t<T, 64, 64, 128>(p, ws, st);
+        if (p.dv == 128) return launch_generic_t<T, 64, 128, 128>(p, ws, st);
+    }
     return GTR_GLA_ERR_CHUNK;
 }
 

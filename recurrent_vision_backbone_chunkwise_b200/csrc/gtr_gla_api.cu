@@ -69,9 +69,11 @@ static bool head_dims_ok(int dk, int dv) {
     return (dk == 64 || dk == 128) && (dv == 64 || dv == 128);
 }
 
-static bool chunk_ok(int dtype, int chunk) {
-    if (dtype == GTR_GLA_F32) return chunk == 32 || chunk == 64;
-    return chunk == 32 || chunk == 64;
+// Chunk lengths: 32 and 64 for every case; 128 with d_k = 64 (the CUDA-core
+// path keeps a chunk's q, k and gates in shared memory, which a 128 x 128
+// chunk would overflow).
+static bool chunk_ok(int chunk, int dk) {
+    return chunk == 32 || chunk == 64 || (chunk == 128 && dk == 64);
 }
 
 static int validate_shape(int B, int H, int gh, int gw, int dk, int dv, int dtype, int chunk) {
@@ -80,7 +82,7 @@ static int validate_shape(int B, int H, int gh, int gw, int dk, int dv, int dtyp
     if (dtype != GTR_GLA_F16 && dtype != GTR_GLA_BF16 && dtype != GTR_GLA_F32)
         return GTR_GLA_ERR_DTYPE;
     if (!head_dims_ok(dk, dv)) return GTR_GLA_ERR_HEAD_DIM;
-    if (!chunk_ok(dtype, chunk)) return GTR_GLA_ERR_CHUNK;
+    if (!chunk_ok(chunk, dk)) return GTR_GLA_ERR_CHUNK;
     return GTR_GLA_OK;
 }
 

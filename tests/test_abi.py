@@ -93,8 +93,12 @@ def test_argument_errors_return_before_launch(gla, kw, code):
     assert call_ex(gla, **kw) == code
 
 
-def test_fp32_chunk_limits(gla):
-    assert call_ex(gla, dtype=gla.F32, chunk=128) == -7
+def test_chunk_128_needs_dk_64(gla):
+    # chunk 128 is supported only with d_k = 64 (shared-memory bound); the
+    # calls below are rejected before anything is launched
+    for dtype in (gla.F16, gla.BF16, gla.F32):
+        assert call_ex(gla, dtype=dtype, chunk=128, dk=128, dv=128) == -7
+        assert call_ex(gla, dtype=dtype, chunk=128, dk=128, dv=64) == -7
 
 
 def test_noalloc_rejects_before_touching_memory(gla):

@@ -93,7 +93,7 @@ def test_1024_b4_stress_gates(direction):
     check(shape, dtype, direction, gates="stress")
 
 
-@pytest.mark.parametrize("chunk", [32, 64])
+@pytest.mark.parametrize("chunk", [32, 64, 128])
 @pytest.mark.parametrize("direction", [0, 3])
 def test_chunk_sweep_16k(chunk, direction):
     shape, dtype = CONFIGS["16k_d64"]
@@ -213,3 +213,10 @@ def test_band_of_extreme_gates(direction):
     ref_o, ref_s = oracle.forward(q, k, v, la, direction)
     assert rel(out, ref_o) <= 5e-3
     assert rel(fs, ref_s) <= 5e-3
+
+
+@pytest.mark.parametrize("direction", [1, 2])
+def test_chunk_128_fp32_ragged(direction):
+    """Chunk 128 on the 640x640 grid: 12 full chunks and a 64-token tail."""
+    shape, _ = CONFIGS["640_b1"]
+    check(shape, "f32", direction, chunk=128)
