@@ -220,3 +220,20 @@ def test_chunk_128_fp32_ragged(direction):
     """Chunk 128 on the 640x640 grid: 12 full chunks and a 64-token tail."""
     shape, _ = CONFIGS["640_b1"]
     check(shape, "f32", direction, chunk=128)
+
+
+@pytest.mark.parametrize("direction", [0, 3])
+def test_bf16_head_dim_128(direction):
+    """bf16 with d = 128: four 64-wide fused launches, the second key half
+    accumulating into the output."""
+    shape = Shape(1, 4, 32, 40, 128, 128)
+    check(shape, "bf16", direction, seed=11)
+
+
+@pytest.mark.parametrize("dims", [(64, 128), (128, 64)])
+def test_rectangular_head_dims_column_scans_edge_grid(dims):
+    """Mixed head sizes on a grid whose height is not a multiple of 8 (the
+    column scans take the row-gather path)."""
+    shape = Shape(1, 3, 13, 9, dims[0], dims[1])
+    for direction in (2, 3):
+        check(shape, "f16", direction, seed=13)
