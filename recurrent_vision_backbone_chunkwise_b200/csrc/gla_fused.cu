@@ -65,6 +65,7 @@ constexpr int kThreads = 32 * (kWarpEpi0 + kEpiWarps);
 constexpr int kOpThreads = 32 * kOpWarps, kEpiThreads = 32 * kEpiWarps;
 constexpr int kBarOp = 1, kBarEpi = 2;  // named barrier ids
 constexpr int kMaxSegments = 64;        // segments per (b,h): bounds the fold
+constexpr int kFoldDepth = 3;           // aggregates in flight during the fold
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kSpanLimit = 80.f;  // max -g (natural log) for the factorised scores
 
@@ -91,6 +92,7 @@ constexpr uint32_t MISC_BYTES = 8192;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory");
 static_assert(MISC_TOT + 2 * kOpWarps * 64 * 4 <= MISC_BYTES, "misc area");
+static_assert(kMaxSegments * 64 * 4 <= 2 * 8192, "the fold stages every gate total in the A buffers");
 static_assert(FC % kOpWarps == 0 && FC / kOpWarps == 8, "operand warps own 8 tokens each");
 
 constexpr uint32_t kTmemCols = 512;
@@ -570,8 +572,9 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
                 gafter.x += g.x;
                 gafter.y += g.y;
                 if (it == npre - 1) {  // the segment's gate totals
+                    // no fence of its own: the arrive (release, CTA scope) orders
+                    // the store before the epilogue's release of the flag
                     if (ow == 0) st2(p.aggg + slot * 64 + p2, gafter);
-                    __threadfence();
                     mbar_arrive(&bar_owpre);
                 }
             } else {
@@ -685,14 +688,17 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
                 st2(dst + j * 64 + i, make_float2(__uint_as_float(r[x]), __uint_as_float(r[x + 1])));
             }
             ok = gwait(epl, kBarEpi, kEpiThreads, &bar_owpre, 0, &s_abort, p.err) && ok;
-            __threadfence();
+            // One release store publishes everything: the stores above (and the
+            // operand warps' gate totals, seen through bar_owpre) precede it
+            // through the CTA barrier, and release is cumulative, so no
+            // per-thread fence is needed.
             named_bar_sync(kBarEpi, kEpiThreads);
-            if (epl && ok) st_release(p.flag + slot, 1);
+            if (epl && ok) st_release(p.flag + kWsFlagStride * slot, 1);
         }
         if (seg > 0) {  // fold the earlier segments' aggregates, nearest first
             if (warp == kWarpEpi0) {
                 bool got = true;
-                for (int j = lane; j < seg; j += 32) got = wait_flag(p.flag + (size_t)bh * p.P + j) && got;
+                for (int j = lane; j < seg; j += 32) got = wait_flag(p.flag + kWsFlagStride * ((size_t)bh * p.P + j)) && got;
                 if (!__all_sync(0xffffffffu, got) && lane == 0) {
                     s_abort = 1;
                     latch_error(p.err, kDevErrTimeout);
@@ -700,44 +706,53 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
             }
             named_bar_sync(kBarEpi, kEpiThreads);
             if (s_abort) ok = false;
+            // The earlier segments' gate totals, copied once (coalesced) into
+            // the A buffers, which stay unused until the first mask.
+            float *sGt = reinterpret_cast<float *>(sm + OFF_A);
+            if (ok)
+                for (int e = tid - 32 * kWarpEpi0; e < seg * 64; e += kEpiThreads)
+                    sGt[e] = __ldcg(p.aggg + (size_t)bh * p.P * 64 + e);
+            named_bar_sync(kBarEpi, kEpiThreads);
             float2 acc[4];  // log-gate sums of the segments between the source and this one
 #pragma unroll
             for (int c = 0; c < 4; ++c) acc[c] = make_float2(0.f, 0.f);
-            // software-pipelined: the next aggregate's loads are in flight
-            // while the current one is folded
-            float2 v[8], gt[4], vn[8], gtn[4];
-            auto load = [&](int d, float2 *vv, float2 *gg) {
-                const size_t src = (size_t)bh * p.P + (seg - 1 - d);
-                const float *ag = p.agg + src * 4096;
+            // software-pipelined: the next kFoldDepth - 1 aggregates' loads are
+            // in flight while one is folded (same summation order as a plain loop)
+            float2 vb[kFoldDepth][8];
+            auto load = [&](int d, float2 *vv) {
+                const float *ag = p.agg + ((size_t)bh * p.P + (seg - 1 - d)) * 4096;
 #pragma unroll
                 for (int x = 0; x < 16; x += 2) {
                     const int j = r0 + 8 * ((x >> 1) & 1), i = hc + 8 * (x >> 2) + cq;
                     vv[x >> 1] = __ldcg(reinterpret_cast<const float2 *>(ag + j * 64 + i));
                 }
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    gg[c] = __ldcg(reinterpret_cast<const float2 *>(p.aggg + src * 64 + hc + 8 * c + cq));
             };
-            if (ok) load(0, v, gt);
-            for (int d = 0; d < seg && ok; ++d) {
-                if (d + 1 < seg) load(d + 1, vn, gtn);
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const float2 sc = ex2_2(acc[c]);
+            for (int e = 0; e < kFoldDepth; ++e)
+                if (ok && e < seg) load(e, vb[e]);
+            for (int d0 = 0; d0 < seg && ok; d0 += kFoldDepth) {
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const int x = 4 * c + 2 * h;
-                        const float2 t = ffma2(sc, v[x >> 1], make_float2(S[x], S[x + 1]));
-                        S[x] = t.x;
-                        S[x + 1] = t.y;
+                for (int e = 0; e < kFoldDepth; ++e) {
+                    const int d = d0 + e;
+                    if (d < seg) {
+                        const float *gt = sGt + (seg - 1 - d) * 64 + hc + cq;
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            const float2 sc = ex2_2(acc[c]);
+#pragma unroll
+                            for (int h = 0; h < 2; ++h) {
+                                const int x = 4 * c + 2 * h;
+                                const float2 t = ffma2(sc, vb[e][x >> 1], make_float2(S[x], S[x + 1]));
+                                S[x] = t.x;
+                                S[x + 1] = t.y;
+                            }
+                            const float2 g2 = ld2(gt + 8 * c);
+                            acc[c].x += g2.x;
+                            acc[c].y += g2.y;
+                        }
+                        if (d + kFoldDepth < seg) load(d + kFoldDepth, vb[e]);
                     }
-                    acc[c].x += gt[c].x;
-                    acc[c].y += gt[c].y;
                 }
-#pragma unroll
-                for (int x = 0; x < 8; ++x) v[x] = vn[x];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) gt[c] = gtn[c];
             }
         }
         // state k^T (tf32) -> rows 64-127 of the B tile of the stage holding chunk k
@@ -874,7 +889,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
     __syncthreads();
     if (s_last) {  // last CTA to finish: leave the workspace ready for the next call
         if (p.P > 1)
-            for (int idx = tid; idx < p.BH * p.P; idx += kThreads) p.flag[idx] = 0;
+            for (int idx = tid; idx < p.BH * p.P; idx += kThreads) p.flag[kWsFlagStride * idx] = 0;
         if (tid == 0) {
             p.ctr[0] = 0;
             p.ctr[1] = 0;

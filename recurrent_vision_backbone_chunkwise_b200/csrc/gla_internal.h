@@ -24,8 +24,12 @@ struct Problem {
 // Every workspace starts with a fixed header that only the fused kernel uses
 // (ticket / completion counters and segment flags).  It is zero before a call
 // and zero after it; the data areas of both paths start after it.
-constexpr size_t kWsHeaderBytes = 4096;
-constexpr int kWsMaxFlags = 960;  // flag slots available in the header
+// Each segment flag has a 128-byte line of its own (kWsFlagStride ints), so a
+// release store never lands on a line that other CTAs are polling for a
+// different flag.
+constexpr size_t kWsHeaderBytes = 65536;
+constexpr int kWsFlagStride = 32;
+constexpr int kWsMaxFlags = (int)((kWsHeaderBytes - 256) / (4 * kWsFlagStride));  // 510
 
 // Record that one kernel was launched (feeds gtr_gla_launch_count()).
 void note_launch();

@@ -155,7 +155,7 @@ def test_final_state_optional_and_out_untouched_elsewhere():
 
 def test_workspace_shared_between_paths_and_left_clean():
     """The CUDA-core path (chunk 32) and the fused path (chunk 64) may share one
-    workspace; the fused kernel's 4 KiB synchronisation header is zero after
+    workspace; the fused kernel's 64 KiB synchronisation header is zero after
     every call."""
     shape, dtype = CONFIGS["640_b1"]
     q, k, v, la = (t.cuda() for t in case(shape, dtype, 0, "normal"))
@@ -167,7 +167,7 @@ def test_workspace_shared_between_paths_and_left_clean():
         out, fs = g.gtr_gla_fwd_ex(q, k, v, la, 3, chunk=chunk, workspace=ws)
         assert g.gtr_gla_status() == 0
         assert rel(out, ref_o) <= TOL[dtype] and rel(fs, ref_s) <= TOL[dtype]
-        assert int(ws[:4096].count_nonzero()) == 0
+        assert int(ws[:65536].count_nonzero()) == 0
 
 
 def test_cuda_graph_replay_matches_eager():
