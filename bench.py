@@ -55,22 +55,42 @@ def workload_bytes(shape, dtype: str) -> int:
             + shape.B * shape.H * shape.d_k * shape.d_v * 4)
 
 
-def profiled_traffic(workload: str):
-    """DRAM bytes of one launch of the fused kernel for `workload`, from the
-    committed ncu summary, if that summary was taken on the current kernel
-    source (its sha256 prefix matches); else None."""
+KERNEL_FILES = ("gla_fused.cu", "sm100.cuh", "gla_common.cuh", "gla_internal.h")
+
+
+def kernel_code_hash() -> str:
+    """sha256 prefix of the fused kernel's code: its source and the headers it
+    includes, with comments and whitespace removed (a comment edit does not
+    make a profile stale; any code change does)."""
     import hashlib
     import re
 
+    h = hashlib.sha256()
+    for name in KERNEL_FILES:
+        with open(os.path.join(ROOT, "recurrent_vision_backbone_chunkwise_b200", "csrc", name)) as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(name.encode() + b"\0" + " ".join(text.split()).encode() + b"\0")
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes of one launch of the fused kernel for `workload`, from the
+    committed ncu summary, if that summary was taken on the current kernel
+    code (kernel_code_hash matches); else None."""
+    import re
+
     prof = os.path.join(ROOT, "profiles", "gla_fused_kernel.md")
-    src = os.path.join(ROOT, "recurrent_vision_backbone_chunkwise_b200", "csrc", "gla_fused.cu")
-    if not (os.path.exists(prof) and os.path.exists(src)):
+    if not os.path.exists(prof):
         return None
     text = open(prof).read()
-    m = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]{16})", text)
-    with open(src, "rb") as f:
-        if not m or hashlib.sha256(f.read()).hexdigest()[:16] != m.group(1):
+    m = re.search(r"kernel_code_sha256_16:\s*([0-9a-f]{16})", text)
+    try:
+        if not m or kernel_code_hash() != m.group(1):
             return None
+    except OSError:
+        return None
     m = re.search(r"traffic_bytes_per_launch\s+" + re.escape(workload) + r"\s+(\d+)", text)
     return int(m.group(1)) if m else None
 

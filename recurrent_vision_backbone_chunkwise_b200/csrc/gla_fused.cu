@@ -5,7 +5,8 @@
 // Dense Prediction" (x-techcon article, section 算子) -- chunks compute their
 // own state contribution in parallel, boundary states are passed along, each
 // chunk's output is produced in parallel, scores stay on chip -- mapped onto
-// one launch of 320-thread CTAs, one per SM:
+// one launch of 576-thread CTAs, one per SM (head sizes of 128 run as four
+// launches of 64-wide parts, see launch_fused):
 //
 //   * a CTA owns a segment of L consecutive 64-token chunks of one (b,h);
 //     CTAs take their segment from a ticket counter, so a segment only ever
@@ -14,7 +15,8 @@
 //     aggregate state contribution, transposed,
 //       A_seg^T = sum_c V_c^T (k_c . e^{G_after(c) + g_c - b_c}),
 //     accumulates in TMEM (chunks visited last to first, every factor <= 1)
-//     and is published with the segment's gate totals;
+//     and is published with the segment's gate totals (one release store of
+//     a flag with a cache line of its own);
 //   * boundary: the incoming state is the fold of every earlier segment's
 //     aggregate, nearest first, S_in = sum_j diag(e^{G(j..seg)}) A_j (a fixed
 //     order: results are bitwise reproducible);
@@ -27,20 +29,22 @@
 //       S      <- diag(e^{g}) S + dS   (fp32, registers of the epilogue warps)
 //
 // Roles (warps):
-//   0      producer: row tables and TMA row gathers of q, k, v, log_alpha into
-//          a 3-stage ring (rows fetched in scan order, so every direction
-//          reads and writes the row-major grid in place);
-//   1      MMA issue (one lane) and TMEM allocation;
-//   2..5   operand warps: gate factors (one exponential per element, running
-//          products), Q^ / K~ (tf32, written over log_alpha / q,k in place)
-//          and K^ (f16/bf16), 16 token rows each;
-//   6..9   epilogue warps, one per TMEM lane quadrant: causal mask, state
-//          update (state in registers, a tf32 copy in shared memory as the
-//          next chunk's MMA operand), output stores, the fold, the
-//          aggregate's publication.
-// Chunk k's scores and dS are issued as soon as its operands are ready, ahead
-// of chunk k-1's output product, so the only serial chain from chunk to chunk
-// is the epilogue's state update.
+//   0       producer: row tables and TMA tile loads (row scans: one box per
+//           tensor; column scans: column slabs, or four-row gathers) of q,
+//           k, v, log_alpha into a 3-stage ring, in scan order, so every
+//           direction reads and writes the row-major grid in place;
+//   1       MMA issue (one lane) and TMEM allocation;
+//   2..9    operand warps, 8 token rows each: gate factors (one exponential
+//           per element, running products), Q^ / K~ (tf32, written over
+//           log_alpha / q,k in place) and K^ (f16/bf16);
+//   10..17  epilogue warps, two per TMEM lane quadrant (32 columns each):
+//           state update (state in registers, a tf32 copy in shared memory
+//           as the next chunk's MMA operand), causal mask, output stores,
+//           the fold, the aggregate's publication.
+// Per chunk k the MMA warp issues A V of chunk k-1 as soon as its mask is in
+// shared memory (this releases that chunk's stage early), then dS of chunk
+// k, then the scores of chunk k once state k is in its stage; the epilogue
+// updates the state, masks chunk k and stores chunk k-1's output.
 //
 // Chunks whose in-chunk gate span exceeds kSpanLimit (e^{-b} would leave fp32
 // range) get their scores from an exact CUDA-core evaluation by the operand

@@ -1,0 +1,70 @@
+"""Host-side pieces of bench.py (CPU only): the kernel-code hash that decides
+whether the committed ncu traffic figures still describe the kernel, and the
+algorithmic byte count of the roofline."""
+import os
+import shutil
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+CSRC = os.path.join("recurrent_vision_backbone_chunkwise_b200", "csrc")
+
+
+@pytest.fixture
+def tree(tmp_path, monkeypatch):
+    """A copy of the kernel sources and the profile summary, with bench.ROOT
+    pointing at it."""
+    os.makedirs(tmp_path / CSRC)
+    for name in bench.KERNEL_FILES:
+        shutil.copy(os.path.join(ROOT, CSRC, name), tmp_path / CSRC / name)
+    os.makedirs(tmp_path / "profiles")
+    shutil.copy(os.path.join(ROOT, "profiles", "gla_fused_kernel.md"), tmp_path / "profiles")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    return tmp_path
+
+
+def _edit(path, fn):
+    with open(path) as f:
+        text = f.read()
+    with open(path, "w") as f:
+        f.write(fn(text))
+
+
+def test_code_hash_ignores_comments_and_whitespace(tree):
+    h0 = bench.kernel_code_hash()
+    _edit(tree / CSRC / "gla_fused.cu", lambda t: "// a new comment line\n" + t.replace("\n", "\n\n", 3))
+    _edit(tree / CSRC / "sm100.cuh", lambda t: t + "\n/* trailing\n block comment */\n")
+    assert bench.kernel_code_hash() == h0
+
+
+@pytest.mark.parametrize("name", ["gla_fused.cu", "sm100.cuh"])
+def test_code_hash_sees_code_changes(tree, name):
+    h0 = bench.kernel_code_hash()
+    _edit(tree / CSRC / name, lambda t: t + "\nconstexpr int kProbe = 1;\n")
+    assert bench.kernel_code_hash() != h0
+
+
+def test_traffic_only_while_the_profile_matches(tree):
+    prof = tree / "profiles" / "gla_fused_kernel.md"
+    _edit(prof, lambda t: "kernel_code_sha256_16: %s\n" % bench.kernel_code_hash() +
+          t.replace("kernel_code_sha256_16", "earlier_hash"))
+    got = bench.profiled_traffic("1024_b4")
+    assert isinstance(got, int) and got > 0
+    assert bench.profiled_traffic("no_such_workload") is None
+    _edit(tree / CSRC / "gla_fused.cu", lambda t: t + "\nconstexpr int kProbe = 2;\n")
+    assert bench.profiled_traffic("1024_b4") is None
+
+
+def test_workload_bytes_per_token_head():
+    """768 B per token-head at d = 64 in fp16 (q, k, v, out at 2 B per element,
+    log_alpha at 4 B), plus the fp32 final state per (b,h)."""
+    from recurrent_vision_backbone_chunkwise_b200.inputs import CONFIGS, Shape
+
+    shape, dtype = CONFIGS["640_b1"]
+    assert bench.workload_bytes(shape, dtype) == 6 * 1600 * 768 + 6 * 64 * 64 * 4
+    s = Shape(1, 1, 2, 3, 128, 64)  # d_k = 128, d_v = 64, fp32
+    assert bench.workload_bytes(s, "f32") == 6 * (128 * 4 * 2 + 64 * 4 + 128 * 4 + 64 * 4) + 128 * 64 * 4
