@@ -38,16 +38,13 @@ void note_launch();
 // (kernel, device): later calls (e.g. inside a stream capture) touch no CUDA API.
 int ensure_smem(const void *func, size_t bytes);
 
-// Encode a [rows][cols] row-gather TMA map (tensormap.cu); 0 on success.
-int encode_rows_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int esize,
-                    uint64_t rows, int cols, bool swizzle128);
-
 // Encode a tiled TMA map of rank 2..5 (tensormap.cu); 0 on success.
 int encode_tile_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int rank,
                     const uint64_t *dims, const uint64_t *strides, const uint32_t *box,
                     bool swizzle128);
 
-// Single-kernel tensor-core path (gla_fused.cu): fp16/bf16, d_k = d_v = 64, chunk 64.
+// Single-kernel tensor-core path (gla_fused.cu): fp16/bf16, chunk 64, d_k and d_v
+// each 64 or 128 (head sizes of 128 as one launch per 64-wide part).
 bool fused_supported(const Problem &p);
 size_t fused_workspace_bytes(const Problem &p);
 int launch_fused(const Problem &p, void *ws, cudaStream_t st);

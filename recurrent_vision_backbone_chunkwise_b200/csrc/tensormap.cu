@@ -23,24 +23,6 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// A 2-D view [rows][cols] of a contiguous row-major tensor, loaded one row
-// per box (TMA row gathers / single-row tiles).  16-bit tensors use the
-// 128-byte swizzle (the tensor-core operand layout); fp32 rows are unswizzled.
-int encode_rows_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int esize,
-                    uint64_t rows, int cols, bool swizzle128) {
-    auto fn = encode_fn();
-    if (!fn) return 1;
-    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)cols * (cuuint64_t)esize};
-    cuuint32_t box[2] = {(cuuint32_t)cols, 1};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? 0 : 1;
-}
-
 // A tiled view of rank 2..5 (dims innermost first, strides in bytes for
 // dims 1..rank-1); loads of `box` elements start at any coordinate, elements
 // outside the tensor read as zero.
