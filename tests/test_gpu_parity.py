@@ -237,3 +237,13 @@ def test_rectangular_head_dims_column_scans_edge_grid(dims):
     shape = Shape(1, 3, 13, 9, dims[0], dims[1])
     for direction in (2, 3):
         check(shape, "f16", direction, seed=13)
+
+
+@pytest.mark.parametrize("direction", [0, 3])
+def test_many_segments_over_several_waves(direction):
+    """B=2, H=20 on the 128x128 grid: the plan splits each (b,h) into 11
+    segments, 440 CTAs in three waves on 148 SMs, with 440 segment flags
+    (one cache line each) in the workspace header.  Later waves fold
+    aggregates published by CTAs that have already exited."""
+    shape = Shape(2, 20, 128, 128, 64, 64)
+    check(shape, "f16", direction, seed=21)
