@@ -42,6 +42,7 @@ from recurrent_vision_backbone_chunkwise_b200.replicas import (  # noqa: E402
 
 METRIC = "GLA fwd tokens/s and µs at 1600/4096/16384 tokens; % of roofline (HBM or TC)"
 L2_BYTES = 126 * 1024 * 1024
+NOMINAL_HBM_GBS = 8000.0  # the ~8 TB/s HBM3e figure the roofline is also quoted against
 DIRECTIONS = (0, 1, 2, 3)
 ESIZE = {"f16": 2, "bf16": 2, "f32": 4}
 
@@ -329,6 +330,18 @@ def main():
     if graph is not None:
         del graph
 
+    # the same calls without graph capture, for comparison (not the headline)
+    eager_ms = call_ms
+    if use_graph:
+        K_eager = min(K, 200)
+        ev_eager = [[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(K_eager)]
+        with torch.cuda.stream(stream):
+            for i in range(K_eager):
+                step(i, ev_eager[i])
+        stream.synchronize()
+        eager_ms = [ev_eager[i][2 * j].elapsed_time(ev_eager[i][2 * j + 1])
+                    for i in range(K_eager) for j in range(len(DIRECTIONS))]
+
     # end-to-end through the public API with pinned host buffers
     K_e2e = min(K, 200)
     host_in = [t.pin_memory() for t in (q0, k0, v0, la0)]
@@ -375,9 +388,12 @@ def main():
                    "cuda_graph": use_graph},
         "kernel_us_per_call": {"mean": 1e6 * mean_call_s,
                                "median": 1e3 * statistics.median(call_ms),
-                               "min": 1e3 * min(call_ms)},
+                               "min": 1e3 * min(call_ms),
+                               "eager_median": 1e3 * statistics.median(eager_ms),
+                               "eager_min": 1e3 * min(eager_ms)},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": profiled_traffic(args.config),
+                     "frac_vs_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
                      "peak_source": f"{peak_kind} copy bandwidth",
                      "bytes_per_call": call_bytes,
                      "timed_unit": "one library call (all kernels of one direction)"},
