@@ -73,7 +73,13 @@ enum {
     GTR_GLA_ERR_WORKSPACE = -8,   /* workspace NULL or smaller than required      */
     GTR_GLA_ERR_CUDA = -9,        /* a CUDA runtime call or launch failed         */
     GTR_GLA_ERR_TIMEOUT = -10,    /* a device-side wait gave up (gtr_gla_status)  */
-    GTR_GLA_ERR_ALIAS = -11       /* out overlaps an input                        */
+    GTR_GLA_ERR_ALIAS = -11,      /* out overlaps an input                        */
+    GTR_GLA_ERR_WORKSPACE_STATE = -12 /* a call found the workspace header not zero
+                                         (calls sharing a workspace overlapped, or it
+                                         was not zero-filled); reported by
+                                         gtr_gla_status, the call did no work in the
+                                         affected segments and the header is clean
+                                         again afterwards                          */
 };
 
 /* ---- entry points --------------------------------------------------- */
@@ -143,7 +149,8 @@ size_t gtr_gla_workspace_size(int B, int H, int grid_h, int grid_w, int d_k, int
 /*
  * gtr_gla_status -- synchronise `stream` and report the first device-side
  * error latched by an earlier call on this device (GTR_GLA_ERR_TIMEOUT when a
- * bounded wait inside a kernel gave up), or GTR_GLA_ERR_CUDA if the stream
+ * bounded wait inside a kernel gave up, GTR_GLA_ERR_WORKSPACE_STATE when a
+ * call found its workspace header not zero), or GTR_GLA_ERR_CUDA if the stream
  * itself reports an error.  Clears the latched error.  Returns GTR_GLA_OK if
  * all is well.
  */

@@ -301,7 +301,13 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
     const size_t slot = (size_t)bh * p.P + seg;
     constexpr uint32_t kFmt = BF16 ? 1u : 0u;
 
-    if (warp == kWarpLoad) {
+    if ((unsigned)ticket >= (unsigned)(p.BH * p.P)) {
+        // A ticket past the last segment means the workspace header was not
+        // zero at launch (two calls sharing it overlapped, or it was never
+        // zeroed): this CTA does no work and reports it; the counters and
+        // flags are still reset below, so the next call starts clean.
+        if (tid == 0) latch_error(p.err, kDevErrWorkspace);
+    } else if (warp == kWarpLoad) {
         // ------------------------------------------------------------ producer
         // TMA tile loads of whole chunks: one box per tensor for row scans,
         // FC / boxh column slabs per tensor for column scans.

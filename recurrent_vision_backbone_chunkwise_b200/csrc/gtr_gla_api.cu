@@ -222,6 +222,7 @@ int gtr_gla_status(cudaStream_t stream) {
     if (host_err != 0 && cudaMemcpyToSymbol(g_dev_err, &zero, sizeof(int)) != cudaSuccess)
         return GTR_GLA_ERR_CUDA;
     if (host_err == kDevErrTimeout) return GTR_GLA_ERR_TIMEOUT;
+    if (host_err == kDevErrWorkspace) return GTR_GLA_ERR_WORKSPACE_STATE;
     return host_err ? GTR_GLA_ERR_CUDA : GTR_GLA_OK;
 }
 
@@ -239,6 +240,8 @@ const char *gtr_gla_strerror(int code) {
         case GTR_GLA_ERR_CUDA: return "CUDA runtime error";
         case GTR_GLA_ERR_TIMEOUT: return "a device-side wait timed out";
         case GTR_GLA_ERR_ALIAS: return "output overlaps an input";
+        case GTR_GLA_ERR_WORKSPACE_STATE:
+            return "workspace header not zero when a call started (overlapping calls sharing it?)";
         default: return "unknown error code";
     }
 }

@@ -50,6 +50,10 @@ def test_strerror_and_count(gla):
     assert gla.gtr_gla_strerror(0) == "ok"
     assert "direction" in gla.gtr_gla_strerror(-4)
     assert gla.gtr_gla_strerror(12345) == "unknown error code"
+    for code in range(-12, 0):  # every declared code has its own text
+        assert gla.gtr_gla_strerror(code) != "unknown error code", code
+    assert "workspace header" in gla.gtr_gla_strerror(-12)
+    assert "timed out" in gla.gtr_gla_strerror(-10)
     assert gla.gtr_gla_launch_count() >= 0
 
 

@@ -247,3 +247,26 @@ def test_many_segments_over_several_waves(direction):
     aggregates published by CTAs that have already exited."""
     shape = Shape(2, 20, 128, 128, 64, 64)
     check(shape, "f16", direction, seed=21)
+
+
+def test_dirty_workspace_header_reports_and_recovers():
+    """A workspace whose ticket counter is not zero at launch (as if two calls
+    sharing it overlapped): one CTA draws a ticket past the last segment and
+    reports GTR_GLA_ERR_WORKSPACE_STATE without touching memory; the segments
+    of the first plane wait for a flag that nothing sets until their bounded
+    wait (about 2 s) gives up.  The call returns, the error is reported, the
+    header is clean again, and the next call on the same workspace is exact."""
+    shape, dtype = CONFIGS["640_b1"]  # 13 segments per (b,h)
+    q, k, v, la = (t.cuda() for t in case(shape, dtype, 0, "normal"))
+    g = gla()
+    need = g.gtr_gla_workspace_size(1, 6, 40, 40, 64, 64, g.F16, 64)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    ws[:4].view(torch.int32)[0] = 1  # ticket counter
+    out, fs = g.gtr_gla_fwd_ex(q, k, v, la, 0, workspace=ws)
+    assert g.gtr_gla_status() == -12  # GTR_GLA_ERR_WORKSPACE_STATE, latched first
+    assert g.gtr_gla_status() == 0   # status clears the latched error
+    assert int(ws[:65536].count_nonzero()) == 0
+    out, fs = g.gtr_gla_fwd_ex(q, k, v, la, 0, workspace=ws)
+    assert g.gtr_gla_status() == 0
+    ref_o, ref_s = reference(shape, dtype, 0, "normal", 0)
+    assert rel(out, ref_o) <= TOL[dtype] and rel(fs, ref_s) <= TOL[dtype]
