@@ -270,3 +270,12 @@ def test_dirty_workspace_header_reports_and_recovers():
     assert g.gtr_gla_status() == 0
     ref_o, ref_s = reference(shape, dtype, 0, "normal", 0)
     assert rel(out, ref_o) <= TOL[dtype] and rel(fs, ref_s) <= TOL[dtype]
+
+
+@pytest.mark.parametrize("direction", [1, 2])
+def test_many_planes_single_segment(direction):
+    """640 (b,h) planes of an 8x8 grid: more planes than segment flags fit in
+    the workspace header, so every plane is one segment (no aggregates, no
+    flags), 640 CTAs in five waves."""
+    shape = Shape(40, 16, 8, 8, 64, 64)
+    check(shape, "f16", direction, seed=23)
