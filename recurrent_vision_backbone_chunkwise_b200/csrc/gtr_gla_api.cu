@@ -109,8 +109,8 @@ static int validate(const Problem &p) {
     return GTR_GLA_OK;
 }
 
-// fp16/bf16 with d_k = d_v = 64 and chunk 64 run the fused tensor-core kernel;
-// everything else (fp32 I/O, other head sizes or chunk lengths) the
+// fp16/bf16 with chunk 64 run the fused tensor-core kernel (head sizes of 128
+// as 64-wide parts); everything else (fp32 I/O, other chunk lengths) the
 // three-phase CUDA-core path.
 static size_t workspace_bytes(const Problem &p) {
     return fused_supported(p) ? fused_workspace_bytes(p) : generic_workspace_bytes(p);
