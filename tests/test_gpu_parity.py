@@ -136,6 +136,25 @@ def test_memoryless_gates_match():
     assert rel(fs, ref_fs) <= 5e-3
 
 
+@pytest.mark.parametrize("dtype", ["f16", "f32"])
+def test_gates_one_is_causal_linear_attention(dtype):
+    """log_alpha = 0 everywhere (no decay, the longest memory): the output is
+    plain causal linear attention tril(Q K^T) V and the final state K^T V,
+    written out with numpy matmuls; 1600 tokens in 13 segments (fp16, fused
+    path) or one CUDA-core scan (fp32)."""
+    shape = Shape(1, 3, 40, 40, 64, 64)
+    q, k, v, _ = make_inputs(shape, dtype, 5)
+    la = torch.zeros(q.shape)
+    g = gla()
+    out, fs = g.gtr_gla_fwd_ex(q.cuda(), k.cuda(), v.cuda(), la.cuda(), 0)
+    assert g.gtr_gla_status() == 0
+    Q, K, V = (t.double().numpy().reshape(1, 3, 1600, 64) for t in (q, k, v))
+    ref_o = np.einsum("bhts,bhsd->bhtd", np.tril(np.einsum("bhtd,bhsd->bhts", Q, K)), V)
+    ref_s = np.einsum("bhti,bhtj->bhij", K, V)
+    assert rel(out.reshape(1, 3, 1600, 64), ref_o) <= TOL[dtype]
+    assert rel(fs, ref_s) <= TOL[dtype]
+
+
 def test_deterministic():
     shape, dtype = CONFIGS["1024_b1"]
     a, sa = run_gpu(shape, dtype, 0, "normal", 2)
