@@ -67,6 +67,37 @@ def make_inputs(shape: Shape, dtype: str = "f16", seed: int = 0, gates: str = "n
             log_alpha.contiguous())
 
 
+def make_swiglu_inputs(B: int, grid_h: int, grid_w: int, C: int, F: int, dtype: str = "f16",
+                       seed: int = 0):
+    """Seeded synthetic input and weights of the Spatial SwiGLU block (no
+    trained weights exist here).  One CPU generator; draw order x, w_gu, b_gu,
+    w_dw, b_dw, w_down, b_down, each randn in fp32, then scaled: x ~ N(0, 1),
+    linear maps ~ N(0, 1/fan_in), biases ~ 0.1 N(0, 1), depthwise taps
+    ~ N(0, 1/9).  x, w_gu, w_down are cast to the I/O dtype (tensor-core
+    operands); biases and depthwise taps stay fp32.  Layouts: x [B, grid_h,
+    grid_w, C], w_gu [2F, C] (gate rows first), b_gu [2F], w_dw [F, 3, 3],
+    b_dw [F], w_down [C, F], b_down [C]."""
+    if dtype not in DTYPES or dtype == "f32":
+        raise ValueError("dtype must be f16 or bf16")
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+
+    def rn(*shape):
+        return torch.randn(shape, generator=g, dtype=torch.float32)
+
+    x = rn(B, grid_h, grid_w, C)
+    w_gu = rn(2 * F, C) / math.sqrt(C)
+    b_gu = 0.1 * rn(2 * F)
+    w_dw = rn(F, 3, 3) / 3.0
+    b_dw = 0.1 * rn(F)
+    w_down = rn(C, F) / math.sqrt(F)
+    b_down = 0.1 * rn(C)
+    dt = DTYPES[dtype]
+    return (x.to(dt).contiguous(), w_gu.to(dt).contiguous(), b_gu.contiguous(),
+            w_dw.contiguous(), b_dw.contiguous(), w_down.to(dt).contiguous(),
+            b_down.contiguous())
+
+
 # The workloads named for this operator: (name, Shape, dtype, directions).
 CONFIGS = {
     "tiny": (Shape(1, 2, 16, 16, 64, 64), "f32"),
