@@ -23,6 +23,8 @@ BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libgtr_gla.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+# cuBLASLt runs the dense projections of the Spatial SwiGLU block
+LINK = ["-lcublasLt", "-Xlinker", "-rpath=/usr/local/cuda/lib64"]
 NVFLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
            "--expt-relaxed-constexpr", "-I", os.path.join(ROOT, "include")]
 
@@ -68,7 +70,7 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
     with ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
         objs = list(ex.map(compile_one, srcs))
     if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < max(os.path.getmtime(o) for o in objs):
-        cmd = [nvcc] + ARCH + ["-shared", "-cudart", "static", "-o", LIB + ".tmp"] + objs
+        cmd = [nvcc] + ARCH + ["-shared", "-cudart", "static", "-o", LIB + ".tmp"] + objs + LINK
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")

@@ -26,7 +26,7 @@ def declared_functions():
     for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
         text = open(h).read()
         text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-        for m in re.finditer(r"\b(gtr_gla_\w+)\s*\(", text):
+        for m in re.finditer(r"\b(gtr_(?:gla|swiglu)_\w+)\s*\(", text):
             names.add(m.group(1))
     return sorted(names)
 
@@ -34,7 +34,8 @@ def declared_functions():
 def test_header_declares_entry_points():
     names = declared_functions()
     for n in ("gtr_gla_fwd", "gtr_gla_fwd_ex", "gtr_gla_workspace_size", "gtr_gla_status",
-              "gtr_gla_strerror", "gtr_gla_release", "gtr_gla_launch_count"):
+              "gtr_gla_strerror", "gtr_gla_release", "gtr_gla_launch_count",
+              "gtr_swiglu_fwd", "gtr_swiglu_workspace_size"):
         assert n in names
 
 
@@ -43,7 +44,9 @@ def test_library_exports_every_declared_symbol(gla):
     for n in declared_functions():
         assert hasattr(lib, n), f"{n} declared in include/ but not exported"
         # the binding forwards under the same name
-        assert hasattr(gla, n), n
+        from recurrent_vision_backbone_chunkwise_b200 import swiglu
+
+        assert hasattr(swiglu if n.startswith("gtr_swiglu_") else gla, n), n
 
 
 def test_strerror_and_count(gla):
@@ -112,3 +115,29 @@ def test_noalloc_rejects_before_touching_memory(gla):
     assert gla._lib.gtr_gla_fwd_noalloc(*args, 1, 2, 4, 4, 128, 128, 0, vp(0)) == -3
     assert gla._lib.gtr_gla_fwd_noalloc(*args, 1, 2, 4, 4, 64, 64, 7, vp(0)) == -4
     assert gla._lib.gtr_gla_fwd_noalloc(vp(0), *args[1:], 1, 2, 4, 4, 64, 64, 0, vp(0)) == -1
+
+
+def test_swiglu_argument_errors_before_launch(gla):
+    """Spatial SwiGLU entry point: every argument error is reported before
+    anything is launched (the fake pointers are never dereferenced)."""
+    import ctypes as C
+
+    from recurrent_vision_backbone_chunkwise_b200 import swiglu
+
+    lib = swiglu._lib
+    p = C.c_void_p(1 << 20)  # 16-byte aligned fake address
+
+    def call(ptrs=None, B=1, gh=4, gw=4, Cc=64, F=256, dtype=gla.F16, ws=p, wsb=1 << 40):
+        ptrs = ptrs or [p] * 8
+        return lib.gtr_swiglu_fwd(*ptrs, B, gh, gw, Cc, F, dtype, ws, wsb, None)
+
+    assert call(ptrs=[p] * 7 + [None]) == -1          # y NULL
+    assert call(B=0) == -2 and call(Cc=60) == -2 and call(F=100) == -2
+    assert call(dtype=gla.F32) == -6
+    assert call(ptrs=[p] * 6 + [C.c_void_p((1 << 20) + 4), p]) == -5   # b_down misaligned
+    assert call(ptrs=[p] * 8) == -11                  # y aliases the inputs
+    q = [C.c_void_p((1 << 20) + (i << 32)) for i in range(8)]
+    assert call(ptrs=q, ws=None) == -8                 # no workspace
+    assert call(ptrs=q, wsb=16) == -8                  # workspace too small
+    assert swiglu.gtr_swiglu_workspace_size(1, 4, 4, 60, 256) == 0
+    assert swiglu.gtr_swiglu_workspace_size(1, 40, 40, 384, 1536) > 1600 * 3 * 1536 * 2
