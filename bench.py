@@ -105,6 +105,137 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
+def measured_tensor_peak():
+    """Dense bf16 (= fp16) tensor-core TFLOP/s for a kernel timed on its own."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    return 1590.0, "fallback"
+
+
+def swiglu_shape(workload: str):
+    """The Spatial SwiGLU block on a workload's grid: C = 64 channels per head
+    of the attention (H x 64) and a hidden width of 4C (the pages give no
+    widths; 4C is the usual MLP ratio)."""
+    shape, dtype = CONFIGS[workload]
+    C = shape.H * 64
+    return shape.B, shape.grid_h, shape.grid_w, C, 4 * C, ("f16" if dtype == "f32" else dtype)
+
+
+def run_swiglu(args):
+    """Spatial SwiGLU leg (not the headline): tokens/s of the whole block, its
+    tensor-core roofline fraction (6 M C F flops of the two projections), the
+    fused kernel's share from the launch list, the fp64 oracle on the host."""
+    import torch
+    from recurrent_vision_backbone_chunkwise_b200 import gla, swiglu
+    from recurrent_vision_backbone_chunkwise_b200.inputs import make_swiglu_inputs
+
+    ri = rank_info()
+    torch.cuda.set_device(ri.local_rank)
+    dev = torch.device("cuda", ri.local_rank)
+    B, gh, gw, C, F, dtype = swiglu_shape(args.config)
+    M = B * gh * gw
+    ins = make_swiglu_inputs(B, gh, gw, C, F, dtype, seed=replica_seed(0, ri.rank))
+    set_bytes = sum(t.numel() * t.element_size() for t in ins) + M * C * 2
+    R = max(2, math.ceil(2 * L2_BYTES / set_bytes))
+    sets = [([t.to(dev) for t in ins], torch.empty_like(ins[0], device=dev)) for _ in range(R)]
+    ws = torch.empty(swiglu.gtr_swiglu_workspace_size(B, gh, gw, C, F, gla._DTYPE_CODE[ins[0].dtype]),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(i, ev=None):
+        t, y = sets[i % R]
+        if ev is not None:
+            ev[0].record(stream)
+        swiglu.gtr_swiglu_fwd(*t, out=y, workspace=ws, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            step(i)
+    stream.synchronize()
+    assert gla.gtr_gla_status(stream) == 0
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)] for _ in range(K)]
+    launches0 = gla.gtr_gla_launch_count()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(K):
+            step(i, evs[i])
+    launches = gla.gtr_gla_launch_count() - launches0
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(ri.local_rank)
+    sampler.start()
+    time.sleep(0.2)
+    torch.cuda.synchronize()
+    t0 = time.time()
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        graph.replay()
+        end.record(stream)
+    torch.cuda.synchronize()
+    t1 = time.time()
+    clocks = sampler.stop(t0, t1)
+    assert gla.gtr_gla_status(stream) == 0
+    elapsed = max_over_ranks(start.elapsed_time(end), device=dev)
+    call_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    del graph
+    # end to end: x in from pinned host memory, y back, every step
+    hx = ins[0].pin_memory()
+    hy = torch.empty_like(ins[0]).pin_memory()
+    K2 = min(K, 200)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(K2):
+            t, y = sets[i % R]
+            t[0].copy_(hx, non_blocking=True)
+            swiglu.gtr_swiglu_fwd(*t, out=y, workspace=ws, stream=stream)
+            hy.copy_(y, non_blocking=True)
+        e1.record(stream)
+    stream.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), device=dev)
+    mean_s = statistics.mean(call_ms) / 1000.0
+    flops = 6.0 * M * C * F
+    peak, peak_kind = measured_tensor_peak()
+    achieved = flops / mean_s / 1e12
+    line = {
+        "metric": "Spatial SwiGLU block tokens/s; % of tensor-core roofline", "value":
+            aggregate_rate(ri.world, K, M, elapsed), "unit": "tokens/s", "n_gpus": ri.world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": elapsed / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": dtype, "data": "synthetic",
+        "config": {"workload": f"swiglu_{args.config}", "B": B, "grid": [gh, gw], "C": C, "F": F,
+                   "l2": f"inputs and weights rotate over {R} sets "
+                         f"({R * set_bytes / 2**20:.0f} MiB > 126 MiB L2)", "cuda_graph": True},
+        "kernel_us_per_call": {"mean": 1e6 * mean_s, "median": 1e3 * statistics.median(call_ms),
+                               "min": 1e3 * min(call_ms)},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "peak_source": f"{peak_kind} dense bf16 burst",
+                     "flops_per_call": flops,
+                     "timed_unit": "one block: two cuBLASLt projections and the fused kernel"},
+        "gpu_launches": int(launches),
+        "e2e": {"value": aggregate_rate(ri.world, K2, M, e2e_ms), "unit": "tokens/s",
+                "h2d_bytes_per_step": M * C * 2, "d2h_bytes_per_step": M * C * 2, "steps": K2},
+        "clocks": clocks,
+    }
+    if ri.rank == 0 and ri.world == 1 and not args.no_cpu_baseline:
+        import oracle.swiglu as osw
+
+        reps, t0 = 0, time.perf_counter()
+        while time.perf_counter() - t0 < 10.0 and reps < 1000:
+            osw.forward(*ins)
+            reps += 1
+        el = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": reps * M / el, "unit": "tokens/s", "cores": os.cpu_count(),
+                                "kind": "oracle",
+                                "sample": f"{reps} forwards of the full block (numpy fp64) in {el:.1f} s"}
+    if ri.rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 class ClockSampler:
     """nvidia-smi clocks / throttle reasons sampled during the timed region."""
 
@@ -249,8 +380,13 @@ def main():
     ap.add_argument("--config", default="640_b1", choices=sorted(CONFIGS))
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--op", default="gla", choices=["gla", "swiglu"],
+                    help="gla: the headline (chunkwise GLA); swiglu: the Spatial SwiGLU block")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.op == "swiglu" and args.impl == "ours":
+        run_swiglu(args)
+        return
 
     if args.impl == "reference":
         run_reference(args)
