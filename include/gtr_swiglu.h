@@ -26,10 +26,11 @@
  *   y       [B, grid_h, grid_w, C]   I/O dtype, must not overlap any input
  * C and F must be multiples of 8 and every pointer 16-byte aligned.  The two
  * projections are dense GEMMs run by cuBLASLt on the tensor cores (fp32
- * accumulation); the biases, the depthwise convolution, the SiLU gate and the
- * product run in this library's own kernel, in fp32, between them.  The
- * projected gate/value and the gated product are kept in the workspace in the
- * I/O dtype.
+ * accumulation); b_g, b_u, b_dw, the depthwise convolution, the SiLU gate and
+ * the product run in this library's own kernel, in fp32, between them; b_down
+ * is rounded once to the I/O dtype and added in fp32 in the down projection's
+ * epilogue.  The projected gate/value and the gated product are kept in the
+ * workspace in the I/O dtype.
  *
  * Return codes are those of gtr_gla.h; GTR_GLA_ERR_CUDA also covers a
  * cuBLASLt failure.  Calls are asynchronous and stream-ordered.
@@ -57,7 +58,9 @@ size_t gtr_swiglu_workspace_size(int B, int grid_h, int grid_w, int C, int F, in
  *              the GPU.
  * Errors: GTR_GLA_ERR_NULL, _SHAPE (B, grid or C, F <= 0, or C, F not
  * multiples of 8), _DTYPE, _ALIGN, _ALIAS, _WORKSPACE, _CUDA; all but the
- * last are reported before anything is launched.
+ * last are reported before anything is launched.  A wait inside the kernel
+ * that runs out of time (it never should) is reported later, by
+ * gtr_gla_status(), as GTR_GLA_ERR_TIMEOUT.
  */
 int gtr_swiglu_fwd(const void *x, const void *w_gu, const float *b_gu, const float *w_dw,
                    const float *b_dw, const void *w_down, const float *b_down, void *y, int B,

@@ -16,6 +16,7 @@
 #include "../../include/gtr_swiglu.h"
 #include "gla_common.cuh"
 #include "gla_internal.h"
+#include "sm100.cuh"
 
 namespace gtr {
 namespace {
@@ -40,56 +41,268 @@ template <> struct Pair<__nv_bfloat16> {
     }
 };
 
-constexpr int kPairs = 32;   // channel pairs per block (64 channels)
-constexpr int kTokens = 8;   // consecutive tokens of one grid row per block
+// ------------------------------------------------- fused depthwise / gate
+//
+// A persistent kernel, one CTA of 16 warps per SM.  Each CTA owns one block of
+// kCh channels for the whole launch (its taps and biases are staged in shared
+// memory once) and one stream of kTH x kTW token tiles: tiles s, s + S,
+// s + 2S, ... over all images, the S CTAs of a channel block taking one stream
+// each.  At any moment the CTAs thus read whole token rows of S neighbouring
+// tiles, and each TMA row is kCh channels (512 bytes) long.
+// Per tile, two TMA loads fill one slot of a kStages-deep ring: the
+// (kTH+2) x (kTW+2) token halo of the value branch u (zero fill outside the
+// grid is the convolution's padding) and the kTH x kTW gate tile g.  The warps
+// form two groups of 8 taking alternate tiles; thread (channel group cg of 8
+// channels, column col) computes a vertical strip of kTH tokens from shared
+// memory, adds the biases, gates and writes h with 16-byte stores.  A warp
+// covers 4 columns x 8 channel groups, so each of its shared-memory reads is
+// four 128-byte rows and each weight read a broadcast.  Each warp counts itself
+// out of a slot when done with it; the group's last warp out issues the loads
+// of the tile kStages further on into it, so no warp waits to refill (and with
+// no separate producer warp, 16 warps leave 128 registers a thread).
+// Every wait is bounded: on a timeout the waiting thread latches
+// kDevErrTimeout and stops, and before the CTA exits one thread waits
+// (bounded) for every copy still in flight.
 
-// h[m, f] = SiLU(g) * (b_dw[f] + sum_{a,c} w_dw[f,a,c] u[y+a-1, x+c-1, f]) with
-// g = gu[m, f] + b_gu[f] and u = gu[., F + f] + b_gu[F + f] (0 off the grid).
-// One thread per (token, channel pair); a block covers 64 channels of 8
-// consecutive tokens of one grid row, so the 3 x 3 neighbourhoods of its
-// tokens overlap in L1.  All arithmetic in fp32.
-template <typename T>
-__global__ void __launch_bounds__(kPairs * kTokens) swiglu_dw_gate_kernel(
-    const T *__restrict__ gu, const float *__restrict__ b_gu, const float *__restrict__ w_dw,
-    const float *__restrict__ b_dw, T *__restrict__ h, int gh, int gw, int F) {
-    __shared__ float s_w[2 * kPairs][9];
-    const int f0 = blockIdx.y * 2 * kPairs;
-    const int tx = threadIdx.x, ty = threadIdx.y, t = ty * kPairs + tx;
-    for (int e = t; e < 2 * kPairs * 9; e += kPairs * kTokens) {
-        const int c = e / 9;
-        s_w[c][e % 9] = (f0 + c < F) ? w_dw[(size_t)(f0 + c) * 9 + e % 9] : 0.f;
+constexpr int kTW = 8, kTH = 4, kCh = 256;
+constexpr int kStages = 4;
+constexpr int kHaloBytes = (kTH + 2) * (kTW + 2) * kCh * 2;  // 30720
+constexpr int kGBytes = kTH * kTW * kCh * 2;                 // 16384
+constexpr int kStageBytes = kHaloBytes + kGBytes;             // 47104
+// Weight rows: taps 0..8, b_g, then the bias of v for each of 16 border
+// cases e = 4 * (top | 2 bottom) + (left | 2 right): b_dw + b_u times the sum
+// of the taps that fall inside the grid there (the zero padding carries no
+// b_u), so that no thread branches on where its token lies.
+constexpr int kWRows = 10 + 16;
+constexpr int kDwThreads = 32 * 16;
+constexpr size_t kDwSmem = (size_t)kStages * kStageBytes + kWRows * kCh * 4 + kStages * 8 + 2 * kStages * 4 + 128;
+static_assert(kHaloBytes % 128 == 0 && kStageBytes % 128 == 0, "stage alignment");
+static_assert(kDwSmem <= 232448, "shared memory per CTA");
+
+// Float index of channel c in weight row r: the 8 channels of group cg are two
+// float4 at (2r)*32 + cg and (2r+1)*32 + cg, so that 32 consecutive groups
+// read 512 contiguous bytes.
+__host__ __device__ __forceinline__ int wslot(int r, int c) {
+    return ((r * 2 + ((c >> 2) & 1)) * 32 + (c >> 3)) * 4 + (c & 3);
+}
+
+__device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, uint64_t *bar, int c0, int c1,
+                                            int c2, int c3) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(sm100::smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(sm100::smem_u32(bar))
+        : "memory");
+}
+
+// Bounded wait on an mbarrier phase with try_wait, which parks the thread in
+// hardware between checks instead of spinning on the issue slots; gives up
+// after about `limit_ns` of wall time.
+__device__ __forceinline__ bool wait_phase(uint64_t *bar, uint32_t parity, uint64_t limit_ns = 2000000000ull) {
+    if (sm100::mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = sm100::global_timer_ns();
+    while (true) {
+        for (int i = 0; i < 16; ++i)
+            if (sm100::mbar_try_wait(bar, parity)) return true;
+        if (sm100::global_timer_ns() - t0 > limit_ns) return false;
     }
-    __syncthreads();
-    const int f = f0 + 2 * tx;
-    const int xblocks = (gw + kTokens - 1) / kTokens;
-    const int row = blockIdx.x / xblocks;  // b * gh + y
-    const int x = (blockIdx.x % xblocks) * kTokens + ty;
-    if (f >= F || x >= gw) return;
-    const int b = row / gh, y = row % gh;
-    const size_t ld = 2 * (size_t)F;  // row length of gu in elements
-    const size_t m = (size_t)row * gw + x;
-    const float2 bg = make_float2(b_gu[f], b_gu[f + 1]);
-    const float2 bu = make_float2(b_gu[F + f], b_gu[F + f + 1]);
-    float2 v = make_float2(b_dw[f], b_dw[f + 1]);
+}
+
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;"
+        : "=l"(d)
+        : "l"(*reinterpret_cast<const uint64_t *>(&a)), "l"(*reinterpret_cast<const uint64_t *>(&b)));
+    return *reinterpret_cast<float2 *>(&d);
+}
+
+__device__ __forceinline__ float tanh_approx(float x) {
+    float y;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// SiLU(g) * v for two lanes: SiLU(g) = g * sigmoid(g) and
+// sigmoid(g) = (1 + tanh(g / 2)) / 2, so one hardware tanh per element (its
+// relative error, about 2^-11, is that of the fp16 rounding of the result).
+__device__ __forceinline__ float2 silu_mul2(float2 g, float2 v) {
+    const float2 half = make_float2(0.5f, 0.5f);
+    const float2 hg = sm100::fmul2(g, half);
+    const float2 t = make_float2(tanh_approx(hg.x), tanh_approx(hg.y));
+    return sm100::fmul2(sm100::ffma2(hg, t, hg), v);  // g/2 * (1 + t) * v
+}
+
+template <typename T>
+__device__ __forceinline__ void unpack8(const uint4 &w, float2 *f) {
+    f[0] = Pair<T>::unpack(w.x);
+    f[1] = Pair<T>::unpack(w.y);
+    f[2] = Pair<T>::unpack(w.z);
+    f[3] = Pair<T>::unpack(w.w);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kDwThreads, 1) swiglu_dw_gate_kernel(
+    const __grid_constant__ CUtensorMap map_u, const __grid_constant__ CUtensorMap map_g,
+    const float *__restrict__ b_gu, const float *__restrict__ w_dw, const float *__restrict__ b_dw,
+    T *__restrict__ h, const float *__restrict__ b_down, T *__restrict__ b_down_io, int *err, int B, int gh,
+    int gw, int F, int C, int cb0, int ncb, int tiles) {
+    using namespace sm100;
+    extern __shared__ uint8_t smem_raw[];
+    // 128-byte aligned base, derived by pointer arithmetic so that every
+    // access below stays a shared-memory access (not a generic one)
+    uint8_t *smem = smem_raw + ((128u - (smem_u32(smem_raw) & 127u)) & 127u);
+    float *sw = reinterpret_cast<float *>(smem + (size_t)kStages * kStageBytes);
+    uint64_t *full = reinterpret_cast<uint64_t *>(sw + kWRows * kCh);
+    int *released = reinterpret_cast<int *>(full + kStages);  // per slot: warps done with it
+    int *last_issued = released + kStages;                      // per slot: last tile loaded, -1 if none
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int cb = cb0 + (int)(blockIdx.x % ncb);
+    const int S = (int)(gridDim.x / ncb), stream = (int)(blockIdx.x / ncb);
+    const int n = stream < tiles ? (tiles - stream + S - 1) / S : 0;
+    const int tiles_w = (gw + kTW - 1) / kTW, tiles_h = (gh + kTH - 1) / kTH;
+    // loads of tile i of this stream into slot i % kStages
+    auto issue = [&](int i) {
+        const int s = i % kStages;
+        const int tile = stream + i * S;
+        const int b = tile / (tiles_w * tiles_h), r = tile % (tiles_w * tiles_h);
+        const int y0 = (r / tiles_w) * kTH, x0 = (r % tiles_w) * kTW;
+        uint8_t *st = smem + (size_t)s * kStageBytes;
+        mbar_arrive_expect_tx(&full[s], kStageBytes);
+        tma_load_4d(st, &map_u, &full[s], F + cb * kCh, x0 - 1, y0 - 1, b);
+        tma_load_4d_pol(st + kHaloBytes, &map_g, &full[s], cb * kCh, x0, y0, b, l2_policy_evict_first());
+        last_issued[s] = i;
+    };
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);  // the issuing thread's arrival with the byte count
+            released[s] = 0;
+            last_issued[s] = -1;
+        }
+        fence_mbar_init();
+        tma_prefetch_desc(&map_u);
+        tma_prefetch_desc(&map_g);
+        for (int i = 0; i < kStages && i < n; ++i) issue(i);
+    }
+    for (int c = threadIdx.x; c < kCh; c += kDwThreads) {
+        const int f = cb * kCh + c;
+        const bool in = f < F;
+        float w[9];
 #pragma unroll
-    for (int a = 0; a < 3; ++a) {
-        const int yy = y + a - 1;
-        if (yy < 0 || yy >= gh) continue;
+        for (int k = 0; k < 9; ++k) {
+            w[k] = in ? w_dw[(size_t)f * 9 + k] : 0.f;
+            sw[wslot(k, c)] = w[k];
+        }
+        const float bu = in ? b_gu[F + f] : 0.f, bd = in ? b_dw[f] : 0.f;
+        sw[wslot(9, c)] = in ? b_gu[f] : 0.f;
+        for (int e = 0; e < 16; ++e) {
+            float inside = 0.f;
 #pragma unroll
-        for (int c = 0; c < 3; ++c) {
-            const int xx = x + c - 1;
-            if (xx < 0 || xx >= gw) continue;
-            const size_t mm = ((size_t)b * gh + yy) * gw + xx;
-            const float2 u = Pair<T>::unpack(*reinterpret_cast<const uint32_t *>(gu + mm * ld + F + f));
-            v.x = fmaf(s_w[2 * tx][3 * a + c], u.x + bu.x, v.x);
-            v.y = fmaf(s_w[2 * tx + 1][3 * a + c], u.y + bu.y, v.y);
+            for (int k = 0; k < 9; ++k) {
+                const int a = k / 3, cc = k % 3;
+                const bool out = (a == 0 && (e & 4)) || (a == 2 && (e & 8)) || (cc == 0 && (e & 1)) ||
+                                 (cc == 2 && (e & 2));
+                if (!out) inside += w[k];
+            }
+            sw[wslot(10 + e, c)] = bd + bu * inside;
         }
     }
-    const float2 g0 = Pair<T>::unpack(*reinterpret_cast<const uint32_t *>(gu + m * ld + f));
-    const float gx = g0.x + bg.x, gy = g0.y + bg.y;
-    const float hx = gx / (1.f + __expf(-gx)) * v.x;
-    const float hy = gy / (1.f + __expf(-gy)) * v.y;
-    *reinterpret_cast<uint32_t *>(h + m * (size_t)F + f) = Pair<T>::pack(hx, hy);
+    if (b_down_io && blockIdx.x == 0)
+        for (int c = threadIdx.x; c < C; c += kDwThreads) b_down_io[c] = static_cast<T>(b_down[c]);
+    __syncthreads();
+
+    // ------------------------------------------------------ consumers
+    const int grp = warp >> 3, wig = warp & 7;
+    const int cg = (wig & 3) * 8 + (lane & 7), col = (wig >> 2) * 4 + (lane >> 3);
+    const int f = cb * kCh + 8 * cg;
+    const float4 *sw4 = reinterpret_cast<const float4 *>(sw);
+    // eight consecutive floats of row r for this thread's channels, as pairs
+    auto wrow = [&](int r, float2 *w) {
+        const float4 lo4 = sw4[(2 * r) * 32 + cg], hi4 = sw4[(2 * r + 1) * 32 + cg];
+        w[0] = make_float2(lo4.x, lo4.y);
+        w[1] = make_float2(lo4.z, lo4.w);
+        w[2] = make_float2(hi4.x, hi4.y);
+        w[3] = make_float2(hi4.z, hi4.w);
+    };
+    for (int i = grp; i < n; i += 2) {
+        const int s = i % kStages;
+        if (!wait_phase(&full[s], (i / kStages) & 1)) {
+            latch_error(err, kDevErrTimeout);
+            break;
+        }
+        const int tile = stream + i * S;
+        const int b = tile / (tiles_w * tiles_h), r = tile % (tiles_w * tiles_h);
+        const int y0 = (r / tiles_w) * kTH, x = (r % tiles_w) * kTW + col;
+        const uint8_t *st = smem + (size_t)s * kStageBytes;
+        if (x < gw && f < F) {
+            // start from the bias of v for the token's border case
+            float2 acc[kTH][4];
+            const int ecol = (x == 0 ? 1 : 0) | (x == gw - 1 ? 2 : 0);
+#pragma unroll
+            for (int j = 0; j < kTH; ++j) {
+                const int y = y0 + j;
+                wrow(10 + ((y == 0 ? 4 : 0) | (y == gh - 1 ? 8 : 0) | ecol), acc[j]);
+            }
+            // sum over taps (a, c): w[a][c] * u[y0 + j + a - 1, x + c - 1]
+#pragma unroll
+            for (int c = 0; c < 3; ++c) {
+                float2 w[3][4];
+#pragma unroll
+                for (int a = 0; a < 3; ++a) wrow(3 * a + c, w[a]);
+#pragma unroll
+                for (int rr = 0; rr < kTH + 2; ++rr) {
+                    const uint4 raw =
+                        *reinterpret_cast<const uint4 *>(st + ((rr * (kTW + 2) + col + c) * kCh + 8 * cg) * 2);
+                    float2 u[4];
+                    unpack8<T>(raw, u);
+#pragma unroll
+                    for (int a = 0; a < 3; ++a) {
+                        const int j = rr - a;
+                        if (j >= 0 && j < kTH) {
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) acc[j][q] = ffma2(w[a][q], u[q], acc[j][q]);
+                        }
+                    }
+                }
+            }
+            float2 bg[4];
+            wrow(9, bg);
+#pragma unroll
+            for (int j = 0; j < kTH; ++j) {
+                const int y = y0 + j;
+                if (y >= gh) break;
+                const uint4 graw =
+                    *reinterpret_cast<const uint4 *>(st + kHaloBytes + ((j * kTW + col) * kCh + 8 * cg) * 2);
+                float2 g[4];
+                unpack8<T>(graw, g);
+                uint32_t o[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float2 hv = silu_mul2(fadd2(g[q], bg[q]), acc[j][q]);
+                    o[q] = Pair<T>::pack(hv.x, hv.y);
+                }
+                const size_t m = ((size_t)b * gh + y) * gw + x;
+                *reinterpret_cast<uint4 *>(h + m * (size_t)F + f) = make_uint4(o[0], o[1], o[2], o[3]);
+            }
+        }
+        // release the slot; the group's last warp to do so refills it at once
+        __syncwarp();
+        if (lane == 0) {
+            __threadfence_block();
+            if (atomicAdd(&released[s], 1) == 7) {
+                released[s] = 0;
+                __threadfence_block();
+                fence_proxy_async_smem();
+                if (i + kStages < n) issue(i + kStages);
+            }
+        }
+    }
+    // no copy may still be landing in shared memory when the CTA exits
+    // (only possible after a timeout above)
+    __syncthreads();
+    if (threadIdx.x == 0)
+        for (int s = 0; s < kStages; ++s)
+            if (last_issued[s] >= 0 && !wait_phase(&full[s], (last_issued[s] / kStages) & 1))
+                latch_error(err, kDevErrTimeout);
 }
 
 // y[m, c] += bias[c] (used only when cuBLASLt takes no fp32 bias in its
@@ -119,7 +332,7 @@ std::mutex g_lt_mu;
 cublasLtHandle_t g_lt[64];
 std::map<std::tuple<int, int, long long, int, int, bool>, LtPlan> g_plans;
 
-// out[M, N] (row-major) = in[M, K] (row-major) . W[N, K]^T (+ bias[N], fp32).
+// out[M, N] (row-major) = in[M, K] (row-major) . W[N, K]^T (+ bias[N], output type).
 // In cuBLASLt's column-major terms: out^T (N x M) = W (N x K) . in^T (K x M),
 // with W stored as a K x N column-major matrix (transposed in the op).
 // Called with g_lt_mu held.
@@ -139,13 +352,10 @@ int lt_plan(int dev, int dtype, long long M, int N, int K, bool bias, LtPlan **o
                        CUBLAS_STATUS_SUCCESS;
     good = good && cublasLtMatmulDescSetAttribute(pl.op, CUBLASLT_MATMUL_DESC_TRANSB, &opN, sizeof(opN)) ==
                        CUBLAS_STATUS_SUCCESS;
-    if (bias) {
+    if (bias) {  // bias vector in the output type
         const cublasLtEpilogue_t epi = CUBLASLT_EPILOGUE_BIAS;
-        const cudaDataType_t bt = CUDA_R_32F;
         good = good && cublasLtMatmulDescSetAttribute(pl.op, CUBLASLT_MATMUL_DESC_EPILOGUE, &epi, sizeof(epi)) ==
                            CUBLAS_STATUS_SUCCESS;
-        good = good && cublasLtMatmulDescSetAttribute(pl.op, CUBLASLT_MATMUL_DESC_BIAS_DATA_TYPE, &bt,
-                                                      sizeof(bt)) == CUBLAS_STATUS_SUCCESS;
     }
     good = good && cublasLtMatrixLayoutCreate(&pl.a, dt, K, N, K) == CUBLAS_STATUS_SUCCESS;
     good = good && cublasLtMatrixLayoutCreate(&pl.b, dt, K, M, K) == CUBLAS_STATUS_SUCCESS;
@@ -167,7 +377,7 @@ int lt_plan(int dev, int dtype, long long M, int N, int K, bool bias, LtPlan **o
     return good ? GTR_GLA_OK : GTR_GLA_ERR_CUDA;
 }
 
-int lt_gemm(int dev, int dtype, long long M, int N, int K, const void *in, const void *w, const float *bias,
+int lt_gemm(int dev, int dtype, long long M, int N, int K, const void *in, const void *w, const void *bias,
             void *out, void *lt_ws, cudaStream_t st) {
     // one lock across the plan lookup, the bias pointer (an attribute of the
     // shared descriptor) and the enqueue
@@ -186,15 +396,16 @@ int lt_gemm(int dev, int dtype, long long M, int N, int K, const void *in, const
 }
 
 struct SwLayout {
-    size_t gu, h, lt, total;
+    size_t gu, h, bd, lt, total;
 };
 
-SwLayout sw_layout(long long M, int F, size_t es) {
+SwLayout sw_layout(long long M, int C, int F, size_t es) {
     auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
     SwLayout l;
     l.gu = 0;
     l.h = up((size_t)M * 2 * F * es);
-    l.lt = up(l.h + (size_t)M * F * es);
+    l.bd = up(l.h + (size_t)M * F * es);
+    l.lt = up(l.bd + (size_t)C * es);
     l.total = l.lt + kLtWorkspace;
     return l;
 }
@@ -211,6 +422,66 @@ int sw_validate_shape(int B, int gh, int gw, int C, int F, int dtype) {
     return GTR_GLA_OK;
 }
 
+int sm_count(int dev) {
+    static int cache[64];
+    if (!cache[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 0;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+// The fused depthwise / gate kernel over the projected [g | u] (token-major,
+// 2F channels per token): two 4-D TMA views (channels, columns, rows, images),
+// one per box shape.
+int launch_dw_gate(int dtype, const void *gu, const float *b_gu, const float *w_dw, const float *b_dw, void *h,
+                   const float *b_down, void *bd, int B, int gh, int gw, int F, int C, cudaStream_t st) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return GTR_GLA_ERR_CUDA;
+    const int sms = sm_count(dev);
+    if (!sms) return GTR_GLA_ERR_CUDA;
+    int *err = nullptr;
+    int rc = error_word(&err);
+    if (rc) return rc;
+    const CUtensorMapDataType dt =
+        dtype == GTR_GLA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    const uint64_t row = 2ull * 2 * F;  // bytes per token
+    const uint64_t dims[4] = {2ull * F, (uint64_t)gw, (uint64_t)gh, (uint64_t)B};
+    const uint64_t strides[3] = {row, row * gw, row * gw * gh};
+    const uint32_t box_u[4] = {kCh, kTW + 2, kTH + 2, 1}, box_g[4] = {kCh, kTW, kTH, 1};
+    CUtensorMap mu, mg;
+    if (encode_tile_map(&mu, gu, dt, 4, dims, strides, box_u, false) ||
+        encode_tile_map(&mg, gu, dt, 4, dims, strides, box_g, false))
+        return GTR_GLA_ERR_CUDA;
+    const long long tiles_ll = (long long)B * ((gh + kTH - 1) / kTH) * ((gw + kTW - 1) / kTW);
+    if (tiles_ll > (1LL << 30)) return GTR_GLA_ERR_SHAPE;
+    const int tiles = (int)tiles_ll;
+    const int ncb_all = (F + kCh - 1) / kCh;
+    auto kern_h = swiglu_dw_gate_kernel<__half>;
+    auto kern_b = swiglu_dw_gate_kernel<__nv_bfloat16>;
+    if ((rc = ensure_smem(dtype == GTR_GLA_BF16 ? (const void *)kern_b : (const void *)kern_h, kDwSmem))) return rc;
+    // one launch per group of at most `sms` channel blocks (a single launch
+    // unless F > kCh * sms); S = sms / ncb CTAs (tile streams) per block
+    for (int cb0 = 0; cb0 < ncb_all; cb0 += sms) {
+        const int ncb = ncb_all - cb0 < sms ? ncb_all - cb0 : sms;
+        int S = sms / ncb;
+        if (S > tiles) S = tiles;
+        const unsigned grid = (unsigned)(ncb * S);
+        if (dtype == GTR_GLA_BF16)
+            kern_b<<<grid, kDwThreads, kDwSmem, st>>>(mu, mg, b_gu, w_dw, b_dw, static_cast<__nv_bfloat16 *>(h),
+                                                      b_down, cb0 == 0 ? static_cast<__nv_bfloat16 *>(bd) : nullptr,
+                                                      err, B, gh, gw, F, C, cb0, ncb, tiles);
+        else
+            kern_h<<<grid, kDwThreads, kDwSmem, st>>>(mu, mg, b_gu, w_dw, b_dw, static_cast<__half *>(h), b_down,
+                                                      cb0 == 0 ? static_cast<__half *>(bd) : nullptr, err, B, gh,
+                                                      gw, F, C, cb0, ncb, tiles);
+        note_launch();
+        if (cudaPeekAtLastError() != cudaSuccess) return GTR_GLA_ERR_CUDA;
+    }
+    return GTR_GLA_OK;
+}
+
 }  // namespace
 }  // namespace gtr
 
@@ -218,7 +489,7 @@ using namespace gtr;
 
 extern "C" size_t gtr_swiglu_workspace_size(int B, int grid_h, int grid_w, int C, int F, int dtype) {
     if (sw_validate_shape(B, grid_h, grid_w, C, F, dtype)) return 0;
-    return sw_layout((long long)B * grid_h * grid_w, F, 2).total;
+    return sw_layout((long long)B * grid_h * grid_w, C, F, 2).total;
 }
 
 extern "C" int gtr_swiglu_fwd(const void *x, const void *w_gu, const float *b_gu, const float *w_dw,
@@ -239,33 +510,23 @@ extern "C" int gtr_swiglu_fwd(const void *x, const void *w_gu, const float *b_gu
         overlap(y, ny, w_dw, (size_t)F * 36) || overlap(y, ny, b_dw, (size_t)F * 4) ||
         overlap(y, ny, b_down, (size_t)C * 4))
         return GTR_GLA_ERR_ALIAS;
-    const SwLayout l = sw_layout(M, F, es);
+    const SwLayout l = sw_layout(M, C, F, es);
     if (!workspace || workspace_bytes < l.total || ((uintptr_t)workspace & 255u)) return GTR_GLA_ERR_WORKSPACE;
     if (overlap(y, ny, workspace, l.total)) return GTR_GLA_ERR_ALIAS;
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return GTR_GLA_ERR_CUDA;
     char *ws = static_cast<char *>(workspace);
-    void *gu = ws + l.gu, *h = ws + l.h, *lt_ws = ws + l.lt;
+    void *gu = ws + l.gu, *h = ws + l.h, *bd = ws + l.bd, *lt_ws = ws + l.lt;
     // 1. [g | u] without biases (the kernel adds them in fp32)
     rc = lt_gemm(dev, dtype, M, 2 * F, C, x, w_gu, nullptr, gu, lt_ws, stream);
     if (rc) return rc;
     // 2. biases, depthwise 3 x 3 on the value branch, SiLU gate, product
-    const int xblocks = (grid_w + kTokens - 1) / kTokens;
-    const dim3 grid((unsigned)((long long)B * grid_h * xblocks), (F + 2 * kPairs - 1) / (2 * kPairs));
-    const dim3 block(kPairs, kTokens);
-    if (dtype == GTR_GLA_BF16)
-        swiglu_dw_gate_kernel<__nv_bfloat16><<<grid, block, 0, stream>>>(
-            static_cast<const __nv_bfloat16 *>(gu), b_gu, w_dw, b_dw, static_cast<__nv_bfloat16 *>(h), grid_h,
-            grid_w, F);
-    else
-        swiglu_dw_gate_kernel<__half><<<grid, block, 0, stream>>>(static_cast<const __half *>(gu), b_gu, w_dw,
-                                                                   b_dw, static_cast<__half *>(h), grid_h,
-                                                                   grid_w, F);
-    note_launch();
-    if (cudaPeekAtLastError() != cudaSuccess) return GTR_GLA_ERR_CUDA;
-    // 3. y = h W_d^T + b_d (bias in the GEMM's epilogue when cuBLASLt takes an
-    //    fp32 bias for these types, else one pass of this library)
-    rc = lt_gemm(dev, dtype, M, C, F, h, w_down, b_down, y, lt_ws, stream);
+    rc = launch_dw_gate(dtype, gu, b_gu, w_dw, b_dw, h, b_down, bd, B, grid_h, grid_w, F, C, stream);
+    if (rc) return rc;
+    // 3. y = h W_d^T + b_d (the bias, copied to the I/O dtype by the kernel
+    //    above, in the GEMM's epilogue; one pass of this library in fp32 if
+    //    cuBLASLt offers no such epilogue)
+    rc = lt_gemm(dev, dtype, M, C, F, h, w_down, bd, y, lt_ws, stream);
     if (rc) {
         rc = lt_gemm(dev, dtype, M, C, F, h, w_down, nullptr, y, lt_ws, stream);
         if (rc) return rc;

@@ -40,6 +40,9 @@ def run(B, gh, gw, C, F, dtype, seed=0):
     (1, 1, 1, 8, 8),          # one token: only the centre tap
     (2, 16, 20, 64, 256),
     (1, 3, 64, 24, 72),       # a wide grid of three rows
+    (1, 9, 1, 16, 64),        # a single column
+    (2, 1024, 1040, 8, 8),    # more token tiles than one grid dimension holds
+    (1, 4, 5, 8, 38400),      # more channel blocks than SMs: one launch per group of blocks
 ])
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
 def test_swiglu_matches_oracle(shape, dtype):
