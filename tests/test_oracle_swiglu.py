@@ -125,6 +125,9 @@ MUTANTS = [
      "up[:, 1:gh + 1, 1:gw + 1, :] = u",
      "up[:, 1:gh + 1, 1:gw + 1, :] = u; up[:, 0] = up[:, gh]; up[:, gh + 1] = up[:, 1]"),
     ("taps transposed", "v += w_dw[:, a, c] * up", "v += w_dw[:, c, a] * up"),
+    ("value bias in the padding",
+     "up = np.zeros((B, gh + 2, gw + 2, F))",
+     "up = np.zeros((B, gh + 2, gw + 2, F)) + b_gu[F:]"),
 ]
 
 
