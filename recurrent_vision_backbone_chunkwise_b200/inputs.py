@@ -98,6 +98,29 @@ def make_swiglu_inputs(B: int, grid_h: int, grid_w: int, C: int, F: int, dtype: 
             b_down.contiguous())
 
 
+
+def make_tail_inputs(B: int, H: int, grid_h: int, grid_w: int, d_v: int, dtype: str = "f16",
+                     seed: int = 0, o_scale: float = 1.0):
+    """Seeded synthetic inputs of the attention's output tail.  One CPU
+    generator; draw order o, z, w, each randn in fp32: o ~ o_scale * N(0, 1)
+    (the attention output, [B, H, grid_h, grid_w, d_v]), z ~ N(0, 1) (the
+    output-gate projection, [B, grid_h, grid_w, H * d_v]), w ~ 1 + 0.1 N(0, 1)
+    (per-head norm weights, [H, d_v], fp32).  o and z are cast to the I/O
+    dtype."""
+    if dtype not in DTYPES or dtype == "f32":
+        raise ValueError("dtype must be f16 or bf16")
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+
+    def rn(*shape):
+        return torch.randn(shape, generator=g, dtype=torch.float32)
+
+    o = o_scale * rn(B, H, grid_h, grid_w, d_v)
+    z = rn(B, grid_h, grid_w, H * d_v)
+    w = 1.0 + 0.1 * rn(H, d_v)
+    dt = DTYPES[dtype]
+    return o.to(dt).contiguous(), z.to(dt).contiguous(), w.contiguous()
+
 # The workloads named for this operator: (name, Shape, dtype, directions).
 CONFIGS = {
     "tiny": (Shape(1, 2, 16, 16, 64, 64), "f32"),
