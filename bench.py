@@ -57,17 +57,18 @@ def workload_bytes(shape, dtype: str) -> int:
 
 
 KERNEL_FILES = ("gla_fused.cu", "sm100.cuh", "gla_common.cuh", "gla_internal.h")
+TAIL_FILES = ("output_tail.cu", "io_pack.cuh", "gla_common.cuh", "gla_internal.h")
 
 
-def kernel_code_hash() -> str:
-    """sha256 prefix of the fused kernel's code: its source and the headers it
+def kernel_code_hash(files=KERNEL_FILES) -> str:
+    """sha256 prefix of a kernel's code: its source and the headers it
     includes, with comments and whitespace removed (a comment edit does not
     make a profile stale; any code change does)."""
     import hashlib
     import re
 
     h = hashlib.sha256()
-    for name in KERNEL_FILES:
+    for name in files:
         with open(os.path.join(ROOT, "recurrent_vision_backbone_chunkwise_b200", "csrc", name)) as f:
             text = f.read()
         text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
@@ -76,19 +77,19 @@ def kernel_code_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str):
-    """DRAM bytes of one launch of the fused kernel for `workload`, from the
-    committed ncu summary, if that summary was taken on the current kernel
-    code (kernel_code_hash matches); else None."""
+def profiled_traffic(workload: str, profile: str = "gla_fused_kernel.md", files=KERNEL_FILES):
+    """DRAM bytes of one launch of a kernel for `workload`, from the committed
+    ncu summary `profiles/<profile>`, if that summary was taken on the current
+    kernel code (kernel_code_hash(files) matches); else None."""
     import re
 
-    prof = os.path.join(ROOT, "profiles", "gla_fused_kernel.md")
+    prof = os.path.join(ROOT, "profiles", profile)
     if not os.path.exists(prof):
         return None
     text = open(prof).read()
     m = re.search(r"kernel_code_sha256_16:\s*([0-9a-f]{16})", text)
     try:
-        if not m or kernel_code_hash() != m.group(1):
+        if not m or kernel_code_hash(files) != m.group(1):
             return None
     except OSError:
         return None
@@ -236,6 +237,122 @@ def run_swiglu(args):
         print(json.dumps(line), flush=True)
 
 
+
+def run_tail(args):
+    """Output-tail leg (not the headline): token-heads/s of the tail on the
+    workload's attention output (B, H, grid, d_v), its HBM roofline fraction
+    (6 d_v bytes per token-head: o and z read, y written), the fp64 oracle on
+    the host."""
+    import torch
+    from recurrent_vision_backbone_chunkwise_b200 import gla, output_tail
+    from recurrent_vision_backbone_chunkwise_b200.inputs import make_tail_inputs
+
+    ri = rank_info()
+    torch.cuda.set_device(ri.local_rank)
+    dev = torch.device("cuda", ri.local_rank)
+    shape, dtype = CONFIGS[args.config]
+    dtype = "f16" if dtype == "f32" else dtype
+    B, H, gh, gw, dv = shape.B, shape.H, shape.grid_h, shape.grid_w, shape.d_v
+    units = B * H * gh * gw  # token-heads per call
+    ins = make_tail_inputs(B, H, gh, gw, dv, dtype, seed=replica_seed(0, ri.rank))
+    call_bytes = 6 * dv * units + H * dv * 4
+    set_bytes = call_bytes
+    R = max(2, math.ceil(2 * L2_BYTES / set_bytes))
+    sets = [([t.to(dev) for t in ins], torch.empty((B, gh, gw, H * dv), dtype=ins[0].dtype, device=dev))
+            for _ in range(R)]
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(i, ev=None):
+        (o, z, w), y = sets[i % R]
+        if ev is not None:
+            ev[0].record(stream)
+        output_tail.gtr_output_tail_fwd(o, z, w, out=y, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            step(i)
+    stream.synchronize()
+    assert gla.gtr_gla_status(stream) == 0
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)] for _ in range(K)]
+    launches0 = gla.gtr_gla_launch_count()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(K):
+            step(i, evs[i])
+    launches = gla.gtr_gla_launch_count() - launches0
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(ri.local_rank)
+    sampler.start()
+    time.sleep(0.2)
+    torch.cuda.synchronize()
+    t0 = time.time()
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        graph.replay()
+        end.record(stream)
+    torch.cuda.synchronize()
+    t1 = time.time()
+    clocks = sampler.stop(t0, t1)
+    assert gla.gtr_gla_status(stream) == 0
+    elapsed = max_over_ranks(start.elapsed_time(end), device=dev)
+    call_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    del graph
+    # end to end: o and z in from pinned host memory, y back, every step
+    ho, hz = ins[0].pin_memory(), ins[1].pin_memory()
+    hy = torch.empty((B, gh, gw, H * dv), dtype=ins[0].dtype).pin_memory()
+    K2 = min(K, 200)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(K2):
+            (o, z, w), y = sets[i % R]
+            o.copy_(ho, non_blocking=True)
+            z.copy_(hz, non_blocking=True)
+            output_tail.gtr_output_tail_fwd(o, z, w, out=y, stream=stream)
+            hy.copy_(y, non_blocking=True)
+        e1.record(stream)
+    stream.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), device=dev)
+    mean_s = statistics.mean(call_ms) / 1000.0
+    peak, peak_kind = measured_peaks()
+    achieved = call_bytes / mean_s / 1e9
+    line = {
+        "metric": "GLA output tail token-heads/s; % of HBM roofline", "value":
+            aggregate_rate(ri.world, K, units, elapsed), "unit": "token-heads/s", "n_gpus": ri.world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": elapsed / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": dtype, "data": "synthetic",
+        "config": {"workload": f"tail_{args.config}", "B": B, "H": H, "grid": [gh, gw], "d_v": dv,
+                   "l2": f"inputs rotate over {R} sets ({R * set_bytes / 2**20:.0f} MiB > 126 MiB L2)",
+                   "cuda_graph": True},
+        "kernel_us_per_call": {"mean": 1e6 * mean_s, "median": 1e3 * statistics.median(call_ms),
+                               "min": 1e3 * min(call_ms)},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak,
+                     "traffic": profiled_traffic(args.config, "output_tail_kernel.md", TAIL_FILES),
+                     "peak_source": peak_kind, "bytes_per_call": call_bytes,
+                     "timed_unit": "one call of output_tail_kernel"},
+        "gpu_launches": int(launches),
+        "e2e": {"value": aggregate_rate(ri.world, K2, units, e2e_ms), "unit": "token-heads/s",
+                "h2d_bytes_per_step": 4 * dv * units, "d2h_bytes_per_step": 2 * dv * units, "steps": K2},
+        "clocks": clocks,
+    }
+    if ri.rank == 0 and ri.world == 1 and not args.no_cpu_baseline:
+        import oracle.output_tail as otail
+
+        reps, t0 = 0, time.perf_counter()
+        while time.perf_counter() - t0 < 10.0 and reps < 1000:
+            otail.forward(*ins)
+            reps += 1
+        el = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": reps * units / el, "unit": "token-heads/s", "cores": os.cpu_count(),
+                                "kind": "oracle",
+                                "sample": f"{reps} calls of the full tail (numpy fp64) in {el:.1f} s"}
+    if ri.rank == 0:
+        print(json.dumps(line), flush=True)
+
 class ClockSampler:
     """nvidia-smi clocks / throttle reasons sampled during the timed region."""
 
@@ -380,12 +497,16 @@ def main():
     ap.add_argument("--config", default="640_b1", choices=sorted(CONFIGS))
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", default="gla", choices=["gla", "swiglu"],
-                    help="gla: the headline (chunkwise GLA); swiglu: the Spatial SwiGLU block")
+    ap.add_argument("--op", default="gla", choices=["gla", "swiglu", "tail"],
+                    help="gla: the headline (chunkwise GLA); swiglu: the Spatial SwiGLU block; "
+                         "tail: the attention's output tail")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.op == "swiglu" and args.impl == "ours":
         run_swiglu(args)
+        return
+    if args.op == "tail" and args.impl == "ours":
+        run_tail(args)
         return
 
     if args.impl == "reference":

@@ -38,7 +38,7 @@ def _nvcc() -> str:
 
 def _newest_dep() -> float:
     deps = glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h"))
-    deps.append(os.path.join(ROOT, "include", "gtr_gla.h"))
+    deps += glob.glob(os.path.join(ROOT, "include", "*.h"))
     deps.append(os.path.abspath(__file__))
     return max(os.path.getmtime(d) for d in deps if os.path.exists(d))
 

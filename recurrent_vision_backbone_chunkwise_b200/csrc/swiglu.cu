@@ -16,30 +16,11 @@
 #include "../../include/gtr_swiglu.h"
 #include "gla_common.cuh"
 #include "gla_internal.h"
+#include "io_pack.cuh"
 #include "sm100.cuh"
 
 namespace gtr {
 namespace {
-
-template <typename T> struct Pair;
-template <> struct Pair<__half> {
-    static __device__ __forceinline__ float2 unpack(uint32_t w) {
-        return __half22float2(*reinterpret_cast<__half2 *>(&w));
-    }
-    static __device__ __forceinline__ uint32_t pack(float a, float b) {
-        __half2 h = __floats2half2_rn(a, b);
-        return *reinterpret_cast<uint32_t *>(&h);
-    }
-};
-template <> struct Pair<__nv_bfloat16> {
-    static __device__ __forceinline__ float2 unpack(uint32_t w) {
-        return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&w));
-    }
-    static __device__ __forceinline__ uint32_t pack(float a, float b) {
-        __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-        return *reinterpret_cast<uint32_t *>(&h);
-    }
-};
 
 // ------------------------------------------------- fused depthwise / gate
 //
@@ -130,14 +111,6 @@ __device__ __forceinline__ float2 silu_mul2(float2 g, float2 v) {
     const float2 hg = sm100::fmul2(g, half);
     const float2 t = make_float2(tanh_approx(hg.x), tanh_approx(hg.y));
     return sm100::fmul2(sm100::ffma2(hg, t, hg), v);  // g/2 * (1 + t) * v
-}
-
-template <typename T>
-__device__ __forceinline__ void unpack8(const uint4 &w, float2 *f) {
-    f[0] = Pair<T>::unpack(w.x);
-    f[1] = Pair<T>::unpack(w.y);
-    f[2] = Pair<T>::unpack(w.z);
-    f[3] = Pair<T>::unpack(w.w);
 }
 
 template <typename T>

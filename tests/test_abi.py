@@ -26,7 +26,7 @@ def declared_functions():
     for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
         text = open(h).read()
         text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-        for m in re.finditer(r"\b(gtr_(?:gla|swiglu)_\w+)\s*\(", text):
+        for m in re.finditer(r"\b(gtr_(?:gla|swiglu|output_tail)_\w+)\s*\(", text):
             names.add(m.group(1))
     return sorted(names)
 
@@ -35,7 +35,7 @@ def test_header_declares_entry_points():
     names = declared_functions()
     for n in ("gtr_gla_fwd", "gtr_gla_fwd_ex", "gtr_gla_workspace_size", "gtr_gla_status",
               "gtr_gla_strerror", "gtr_gla_release", "gtr_gla_launch_count",
-              "gtr_swiglu_fwd", "gtr_swiglu_workspace_size"):
+              "gtr_swiglu_fwd", "gtr_swiglu_workspace_size", "gtr_output_tail_fwd"):
         assert n in names
 
 
@@ -44,9 +44,10 @@ def test_library_exports_every_declared_symbol(gla):
     for n in declared_functions():
         assert hasattr(lib, n), f"{n} declared in include/ but not exported"
         # the binding forwards under the same name
-        from recurrent_vision_backbone_chunkwise_b200 import swiglu
+        from recurrent_vision_backbone_chunkwise_b200 import output_tail, swiglu
 
-        assert hasattr(swiglu if n.startswith("gtr_swiglu_") else gla, n), n
+        mod = swiglu if n.startswith("gtr_swiglu_") else output_tail if n.startswith("gtr_output_tail_") else gla
+        assert hasattr(mod, n), n
 
 
 def test_strerror_and_count(gla):
@@ -141,3 +142,25 @@ def test_swiglu_argument_errors_before_launch(gla):
     assert call(ptrs=q, wsb=16) == -8                  # workspace too small
     assert swiglu.gtr_swiglu_workspace_size(1, 4, 4, 60, 256) == 0
     assert swiglu.gtr_swiglu_workspace_size(1, 40, 40, 384, 1536) > 1600 * 3 * 1536 * 2
+
+
+def test_output_tail_argument_errors_before_launch(gla):
+    """Output-tail entry point: every argument error is reported before
+    anything is launched (the fake pointers are never dereferenced)."""
+    import ctypes as C
+
+    from recurrent_vision_backbone_chunkwise_b200 import output_tail
+
+    lib = output_tail._lib
+    q = [C.c_void_p((1 << 20) + (i << 32)) for i in range(4)]  # distinct, 16-byte aligned
+
+    def call(ptrs=None, B=1, H=2, gh=4, gw=4, dv=64, eps=1e-5, dtype=gla.F16):
+        return lib.gtr_output_tail_fwd(*(ptrs or q), B, H, gh, gw, dv, eps, dtype, None)
+
+    assert call(ptrs=q[:3] + [None]) == -1              # y NULL
+    assert call(B=0) == -2 and call(H=-1) == -2 and call(gw=0) == -2
+    assert call(eps=-1.0) == -2 and call(eps=float("nan")) == -2 and call(eps=float("inf")) == -2
+    assert call(dv=32) == -3 and call(dv=96) == -3
+    assert call(dtype=gla.F32) == -6
+    assert call(ptrs=q[:2] + [C.c_void_p((1 << 20) + (2 << 32) + 8), q[3]]) == -5   # w misaligned
+    assert call(ptrs=q[:3] + [q[0]]) == -11              # y is o
