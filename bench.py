@@ -124,6 +124,30 @@ def swiglu_shape(workload: str):
     return shape.B, shape.grid_h, shape.grid_w, C, 4 * C, ("f16" if dtype == "f32" else dtype)
 
 
+def smi_index(local: int) -> int:
+    """nvidia-smi index of this rank's GPU (the first visible device)."""
+    first = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")[0]
+    return int(first) if first.isdigit() else local
+
+
+def dist_setup(ri, dev):
+    """One NCCL process group over the ranks of a torchrun launch (None when
+    the job has one rank)."""
+    if ri.world <= 1:
+        return None
+    from datetime import timedelta
+
+    import torch.distributed as dist
+
+    dist.init_process_group("nccl", timeout=timedelta(seconds=180), device_id=dev)
+    return dist
+
+
+def dist_barrier(dist):
+    if dist is not None:
+        dist.barrier()
+
+
 def run_swiglu(args):
     """Spatial SwiGLU leg (not the headline): tokens/s of the whole block, its
     tensor-core roofline fraction (6 M C F flops of the two projections), the
@@ -135,6 +159,7 @@ def run_swiglu(args):
     ri = rank_info()
     torch.cuda.set_device(ri.local_rank)
     dev = torch.device("cuda", ri.local_rank)
+    dist = dist_setup(ri, dev)
     B, gh, gw, C, F, dtype = swiglu_shape(args.config)
     M = B * gh * gw
     ins = make_swiglu_inputs(B, gh, gw, C, F, dtype, seed=replica_seed(0, ri.rank))
@@ -167,9 +192,10 @@ def run_swiglu(args):
             step(i, evs[i])
     launches = gla.gtr_gla_launch_count() - launches0
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    sampler = ClockSampler(ri.local_rank)
+    sampler = ClockSampler(smi_index(ri.local_rank))
     sampler.start()
     time.sleep(0.2)
+    dist_barrier(dist)
     torch.cuda.synchronize()
     t0 = time.time()
     with torch.cuda.stream(stream):
@@ -178,6 +204,7 @@ def run_swiglu(args):
         end.record(stream)
     torch.cuda.synchronize()
     t1 = time.time()
+    dist_barrier(dist)
     clocks = sampler.stop(t0, t1)
     assert gla.gtr_gla_status(stream) == 0
     elapsed = max_over_ranks(start.elapsed_time(end), device=dev)
@@ -188,6 +215,7 @@ def run_swiglu(args):
     hy = torch.empty_like(ins[0]).pin_memory()
     K2 = min(K, 200)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist_barrier(dist)
     with torch.cuda.stream(stream):
         e0.record(stream)
         for i in range(K2):
@@ -235,7 +263,8 @@ def run_swiglu(args):
                                 "sample": f"{reps} forwards of the full block (numpy fp64) in {el:.1f} s"}
     if ri.rank == 0:
         print(json.dumps(line), flush=True)
-
+    if dist is not None:
+        dist.destroy_process_group()
 
 
 def run_tail(args):
@@ -250,6 +279,7 @@ def run_tail(args):
     ri = rank_info()
     torch.cuda.set_device(ri.local_rank)
     dev = torch.device("cuda", ri.local_rank)
+    dist = dist_setup(ri, dev)
     shape, dtype = CONFIGS[args.config]
     dtype = "f16" if dtype == "f32" else dtype
     B, H, gh, gw, dv = shape.B, shape.H, shape.grid_h, shape.grid_w, shape.d_v
@@ -284,9 +314,10 @@ def run_tail(args):
             step(i, evs[i])
     launches = gla.gtr_gla_launch_count() - launches0
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    sampler = ClockSampler(ri.local_rank)
+    sampler = ClockSampler(smi_index(ri.local_rank))
     sampler.start()
     time.sleep(0.2)
+    dist_barrier(dist)
     torch.cuda.synchronize()
     t0 = time.time()
     with torch.cuda.stream(stream):
@@ -295,6 +326,7 @@ def run_tail(args):
         end.record(stream)
     torch.cuda.synchronize()
     t1 = time.time()
+    dist_barrier(dist)
     clocks = sampler.stop(t0, t1)
     assert gla.gtr_gla_status(stream) == 0
     elapsed = max_over_ranks(start.elapsed_time(end), device=dev)
@@ -305,6 +337,7 @@ def run_tail(args):
     hy = torch.empty((B, gh, gw, H * dv), dtype=ins[0].dtype).pin_memory()
     K2 = min(K, 200)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist_barrier(dist)
     with torch.cuda.stream(stream):
         e0.record(stream)
         for i in range(K2):
@@ -352,6 +385,9 @@ def run_tail(args):
                                 "sample": f"{reps} calls of the full tail (numpy fp64) in {el:.1f} s"}
     if ri.rank == 0:
         print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
 
 class ClockSampler:
     """nvidia-smi clocks / throttle reasons sampled during the timed region."""
@@ -580,9 +616,7 @@ def main():
 
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
-    gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[0]) \
-        if os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")[0].isdigit() else local
-    sampler = ClockSampler(gpu_index)
+    sampler = ClockSampler(smi_index(local))
     sampler.start()
     time.sleep(0.2)
     if world > 1:

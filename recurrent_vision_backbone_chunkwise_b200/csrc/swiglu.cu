@@ -278,8 +278,9 @@ __global__ void __launch_bounds__(kDwThreads, 1) swiglu_dw_gate_kernel(
                 latch_error(err, kDevErrTimeout);
 }
 
-// y[m, c] += bias[c] (used only when cuBLASLt takes no fp32 bias in its
-// epilogue for these types).
+// y[m, c] += bias[c] in fp32: the fallback for a cuBLASLt that offers no
+// bias epilogue for this GEMM (on B200 with these types it does, and this
+// kernel does not run).
 template <typename T>
 __global__ void add_bias_kernel(T *y, const float *bias, size_t M, int C) {
     const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;  // pair index
