@@ -121,6 +121,51 @@ def make_tail_inputs(B: int, H: int, grid_h: int, grid_w: int, d_v: int, dtype: 
     dt = DTYPES[dtype]
     return o.to(dt).contiguous(), z.to(dt).contiguous(), w.contiguous()
 
+
+def make_backbone_params(C: int, F: int, n_layers: int, dtype: str = "f16", seed: int = 0):
+    """Seeded synthetic weights of n_layers backbone layers (no trained weights
+    exist here).  One CPU generator; per layer, in this order, each randn in
+    fp32 then scaled: ln1_w, ln1_b, w_q, w_k, w_v, w_a, b_a, w_z, w_n, w_o,
+    ln2_w, ln2_b, then the Spatial SwiGLU weights as make_swiglu_inputs draws
+    them (w_gu, b_gu, w_dw, b_dw, w_down, b_down).  LayerNorm weights
+    1 + 0.1 N(0, 1) and biases 0.1 N(0, 1); linear maps N(0, 1/fan_in); gate
+    bias b_a ~ N(0, 1); norm weights w_n ~ 1 + 0.1 N(0, 1).  The projection
+    matrices are in the I/O dtype (tensor-core operands), the rest fp32.
+    Shapes: see oracle/backbone.py."""
+    if dtype not in DTYPES or dtype == "f32":
+        raise ValueError("dtype must be f16 or bf16")
+    if C % 64:
+        raise ValueError("C must be a multiple of 64")
+    H = C // 64
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    dt = DTYPES[dtype]
+
+    def rn(*shape):
+        return torch.randn(shape, generator=g, dtype=torch.float32)
+
+    layers = []
+    for _ in range(n_layers):
+        p = {}
+        p["ln1_w"] = 1.0 + 0.1 * rn(C)
+        p["ln1_b"] = 0.1 * rn(C)
+        for name in ("w_q", "w_k", "w_v", "w_a"):
+            p[name] = (rn(H * 64, C) / math.sqrt(C)).to(dt)
+        p["b_a"] = rn(H * 64)
+        p["w_z"] = (rn(H * 64, C) / math.sqrt(C)).to(dt)
+        p["w_n"] = 1.0 + 0.1 * rn(H, 64)
+        p["w_o"] = (rn(C, H * 64) / math.sqrt(H * 64)).to(dt)
+        p["ln2_w"] = 1.0 + 0.1 * rn(C)
+        p["ln2_b"] = 0.1 * rn(C)
+        p["w_gu"] = (rn(2 * F, C) / math.sqrt(C)).to(dt)
+        p["b_gu"] = 0.1 * rn(2 * F)
+        p["w_dw"] = rn(F, 3, 3) / 3.0
+        p["b_dw"] = 0.1 * rn(F)
+        p["w_down"] = (rn(C, F) / math.sqrt(F)).to(dt)
+        p["b_down"] = 0.1 * rn(C)
+        layers.append({k: v.contiguous() for k, v in p.items()})
+    return layers
+
 # The workloads named for this operator: (name, Shape, dtype, directions).
 CONFIGS = {
     "tiny": (Shape(1, 2, 16, 16, 64, 64), "f32"),
