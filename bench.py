@@ -364,7 +364,7 @@ def run_tail(args):
                                "min": 1e3 * min(call_ms)},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak,
-                     "traffic": profiled_traffic(args.config, "output_tail_kernel.md", TAIL_FILES),
+                     "traffic": profiled_traffic(args.config, "output_tail_kernel_1024_b4.md", TAIL_FILES),
                      "peak_source": peak_kind, "bytes_per_call": call_bytes,
                      "timed_unit": "one call of output_tail_kernel"},
         "gpu_launches": int(launches),
