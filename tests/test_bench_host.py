@@ -68,3 +68,43 @@ def test_workload_bytes_per_token_head():
     assert bench.workload_bytes(shape, dtype) == 6 * 1600 * 768 + 6 * 64 * 64 * 4
     s = Shape(1, 1, 2, 3, 128, 64)  # d_k = 128, d_v = 64, fp32
     assert bench.workload_bytes(s, "f32") == 6 * (128 * 4 * 2 + 64 * 4 + 128 * 4 + 64 * 4) + 128 * 64 * 4
+
+
+def test_tail_traffic_follows_its_own_code_hash(tmp_path, monkeypatch):
+    """The output tail's profile is gated by the hash of its own sources, not
+    by the attention kernel's."""
+    os.makedirs(tmp_path / CSRC)
+    for name in set(bench.TAIL_FILES) | set(bench.KERNEL_FILES):
+        shutil.copy(os.path.join(ROOT, CSRC, name), tmp_path / CSRC / name)
+    os.makedirs(tmp_path / "profiles")
+    prof = "output_tail_kernel_1024_b4.md"
+    shutil.copy(os.path.join(ROOT, "profiles", prof), tmp_path / "profiles")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    got = bench.profiled_traffic("1024_b4", prof, bench.TAIL_FILES)
+    assert isinstance(got, int) and got > 0
+    _edit(tmp_path / CSRC / "gla_fused.cu", lambda t: t + "\nconstexpr int kProbe = 3;\n")
+    assert bench.profiled_traffic("1024_b4", prof, bench.TAIL_FILES) == got
+    _edit(tmp_path / CSRC / "output_tail.cu", lambda t: t + "\nconstexpr int kProbe = 4;\n")
+    assert bench.profiled_traffic("1024_b4", prof, bench.TAIL_FILES) is None
+
+
+def test_swiglu_widths_follow_the_attention_workload():
+    """C = 64 channels per head of the workload, F = 4C, fp16 for the fp32 case."""
+    assert bench.swiglu_shape("1024_b4") == (4, 64, 64, 768, 3072, "f16")
+    assert bench.swiglu_shape("640_b1") == (1, 40, 40, 384, 1536, "f16")
+    assert bench.swiglu_shape("tiny")[-1] == "f16"
+
+
+def test_nvidia_smi_index_and_single_rank_group(monkeypatch):
+    monkeypatch.setenv("CUDA_VISIBLE_DEVICES", "5,6")
+    assert bench.smi_index(1) == 5
+    monkeypatch.setenv("CUDA_VISIBLE_DEVICES", "GPU-1234")
+    assert bench.smi_index(1) == 1
+    monkeypatch.delenv("CUDA_VISIBLE_DEVICES")
+    assert bench.smi_index(3) == 3
+
+    class One:
+        world = 1
+
+    assert bench.dist_setup(One(), None) is None
+    bench.dist_barrier(None)  # a no-op without a group
