@@ -7,6 +7,8 @@ Each pin is independent of the oracle's code:
 - torch autograd through the brute-force quadratic form (explicit gate
   products, scan orders listed position by position);
 - the final-state gradient entering the same way.
+The chunked reorganisation of the gradients (oracle.backward.chunkwise_backward)
+is checked against them for many chunk lengths.
 Planted mistakes in a copy of the oracle must fail them (the last tests).
 """
 import os
@@ -116,6 +118,21 @@ def test_autograd_of_the_quadratic_form(direction):
     for got, ref in zip(grads, (tq.grad, tk.grad, tv.grad, tla.grad)):
         assert np.allclose(got, ref.numpy(), rtol=1e-12, atol=1e-12)
 
+
+
+@pytest.mark.parametrize("direction", [0, 1, 2, 3])
+@pytest.mark.parametrize("chunk", [1, 5, 16, 64, 1000])
+def test_chunkwise_backward_equals_the_token_backward(direction, chunk):
+    """The chunked reorganisation (boundary states, reverse scan of the state
+    gradients, per-chunk matrix products, log-gates through the cumulative
+    sum) gives the token-by-token gradients for any chunk length, including
+    ones that do not divide the token count and one longer than the scan."""
+    q, k, v, la, dO, dS = _case(B=2, H=1, gh=5, gw=7, dk=3, dv=4, seed=30 + direction)
+    for state in (None, dS):
+        ref = ob.backward(q, k, v, la, dO, direction, state)
+        got = ob.chunkwise_backward(q, k, v, la, dO, direction, chunk, state)
+        for a, b in zip(got, ref):
+            assert np.max(np.abs(a - b)) <= 1e-12 * np.max(np.abs(b))
 
 # Planted mistakes: (name, original text, replacement); each original must
 # occur once in oracle/gla_backward.c.
