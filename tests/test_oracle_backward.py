@@ -116,7 +116,11 @@ def test_autograd_of_the_quadratic_form(direction):
     loss.backward()
     grads = ob.backward(q, k, v, la, dO, direction, dS)
     for got, ref in zip(grads, (tq.grad, tk.grad, tv.grad, tla.grad)):
-XX, [1, 5, 16, 64, 1000])
+        assert np.allclose(got, ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("direction", [0, 1, 2, 3])
+@pytest.mark.parametrize("chunk", [1, 5, 16, 64, 1000])
 def test_chunkwise_backward_equals_the_token_backward(direction, chunk):
     """The chunked reorganisation (boundary states, reverse scan of the state
     gradients, per-chunk matrix products, log-gates through the cumulative
