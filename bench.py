@@ -454,14 +454,43 @@ class ClockSampler:
                 "samples": len(window), "window": scope}
 
 
-def cpu_oracle_rate(shape, dtype, seconds: float = 10.0, max_reps: int = 100000):
-    """The fp64 oracle, as it stands, on this host: tokens/s over the four
-    directions of one batch, repeated until ~`seconds` of CPU work."""
+def image_tokens(shape) -> int:
+    """Image tokens of one call: B * grid_h * grid_w (every head of a token is
+    in the same call, so heads are not counted again)."""
+    return shape.B * shape.tokens
+
+
+def oracle_sample(shape, dtype, seconds: float):
+    """Inputs of a bounded CPU sample of `shape`: the grid is cut to its first
+    rows so that one direction of every plane takes about `seconds` / 4 on
+    all host cores (the whole grid when that fits)."""
+    import numpy as np
+
     import oracle
 
-    q, k, v, la = make_inputs(shape, dtype, seed=0)
-    q, k, v, la = (t.double().numpy() for t in (q, k, v, la))
+    q, k, v, la = (t.double().numpy() for t in make_inputs(shape, dtype, seed=0))
     cores = oracle.max_threads()
+    rows = shape.grid_h
+    probe = max(1, min(rows, 8))
+    t0 = time.perf_counter()
+    oracle.forward(*(np.ascontiguousarray(a[:, :, :probe]) for a in (q, k, v, la)), 0,
+                   n_threads=cores)
+    per_row = (time.perf_counter() - t0) / probe
+    rows = max(1, min(rows, int(seconds / 4.0 / max(per_row, 1e-9))))
+    return tuple(np.ascontiguousarray(a[:, :, :rows]) for a in (q, k, v, la)), rows
+
+
+def cpu_oracle_rate(shape, dtype, seconds: float = 10.0, threads=None, max_reps: int = 100000):
+    """The fp64 oracle, as it stands, on this host: image tokens/s over the four
+    directions of a bounded sample of the workload (its first grid rows, all
+    planes), repeated until ~`seconds` of CPU work.  `threads` = OpenMP
+    threads (all host cores by default); the oracle runs one (b,h) plane per
+    thread, so at most B*H of them do work."""
+    import oracle
+
+    (q, k, v, la), rows = oracle_sample(shape, dtype, seconds if threads != 1 else seconds / 8)
+    cores = oracle.max_threads() if threads is None else int(threads)
+    used = min(cores, shape.B * shape.H)
     reps = 0
     t0 = time.perf_counter()
     while True:
@@ -471,57 +500,193 @@ def cpu_oracle_rate(shape, dtype, seconds: float = 10.0, max_reps: int = 100000)
         el = time.perf_counter() - t0
         if el >= seconds or reps >= max_reps:
             break
-    tokens = reps * len(DIRECTIONS) * shape.B * shape.H * shape.tokens
-    return tokens / el, cores, reps, el
+    tokens = reps * len(DIRECTIONS) * shape.B * rows * shape.grid_w
+    sample = (f"{reps} steps x 4 directions of all {shape.B * shape.H} planes on the first "
+              f"{rows} of {shape.grid_h} grid rows in {el:.1f} s, {cores} OpenMP threads "
+              f"({used} busy: one plane per thread)")
+    return {"value": tokens / el, "unit": "tokens/s", "cores": used, "threads": cores,
+            "kind": "oracle", "sample": sample}
+
+
+def workload_config(name: str, world: int, chunk: int = 64) -> dict:
+    """The `config` object of a bench line; both arms print the same one."""
+    shape, dtype = CONFIGS[name]
+    in_bytes = shape.B * shape.H * shape.tokens * (
+        (2 * shape.d_k + shape.d_v) * ESIZE[dtype] + 4 * shape.d_k)
+    set_bytes = in_bytes + len(DIRECTIONS) * shape.B * shape.H * shape.tokens * shape.d_v * ESIZE[dtype]
+    R = max(2, math.ceil(2 * L2_BYTES / set_bytes))
+    return {"workload": name, "B": shape.B, "H": shape.H, "grid": [shape.grid_h, shape.grid_w],
+            "tokens": shape.tokens, "d_k": shape.d_k, "d_v": shape.d_v, "io_dtype": dtype,
+            "chunk": chunk, "directions": 4,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": f"inputs rotate over {R} buffer sets "
+                  f"({R * set_bytes / 2**20:.0f} MiB > 126 MiB L2)"}
 
 
 def run_reference(args):
     """The oracle as the reference arm: exactly `--steps` timed steps after
     `--warmup` untimed ones, each step one scan direction (cycling) of every
     (b,h) plane of the workload's grid cut to its first rows, so that the whole
-    run takes about a minute of host time; tokens/s counts the tokens the
-    sample holds."""
+    run takes about a minute of host time; tokens/s counts the image tokens
+    the sample holds."""
     if rank_info().rank != 0:
         return
-    import numpy as np
-
     import oracle
 
     shape, dtype = CONFIGS[args.config]
-    q, k, v, la = (t.double().numpy() for t in make_inputs(shape, dtype, seed=0))
-    cores = oracle.max_threads()
-    t0 = time.perf_counter()
-    oracle.forward(q, k, v, la, 0, n_threads=cores)
-    t_full = time.perf_counter() - t0
     budget = 60.0 / (args.steps + args.warmup)  # seconds of host time per step
-    rows = max(1, min(shape.grid_h, int(shape.grid_h * budget / max(t_full, 1e-9))))
-    qs, ks, vs, las = (np.ascontiguousarray(a[:, :, :rows]) for a in (q, k, v, la))
+    (qs, ks, vs, las), rows = oracle_sample(shape, dtype, 4.0 * budget)
+    cores = oracle.max_threads()
     for i in range(args.warmup):
         oracle.forward(qs, ks, vs, las, DIRECTIONS[i % 4], n_threads=cores)
     t0 = time.perf_counter()
     for i in range(args.steps):
         oracle.forward(qs, ks, vs, las, DIRECTIONS[i % 4], n_threads=cores)
     el = time.perf_counter() - t0
-    tokens = shape.B * shape.H * rows * shape.grid_w
+    tokens = shape.B * rows * shape.grid_w
     rate = args.steps * tokens / el
+    used = min(cores, shape.B * shape.H)
     sample = (f"{args.steps} steps, each one direction of all {shape.B * shape.H} planes "
-              f"on the first {rows} of {shape.grid_h} grid rows ({tokens} tokens), {el:.1f} s")
+              f"on the first {rows} of {shape.grid_h} grid rows ({tokens} image tokens), "
+              f"{el:.1f} s, {cores} OpenMP threads ({used} busy: one plane per thread)")
     line = {
         "impl": "reference", "metric": METRIC, "value": rate, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1000.0 * el / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": args.config, "B": shape.B, "H": shape.H,
-                                        "grid": [shape.grid_h, shape.grid_w],
-                                        "d_k": shape.d_k, "d_v": shape.d_v,
-                                        "io_dtype": dtype, "directions": 4},
-        "cpu_baseline": {"value": rate, "unit": "tokens/s",
-                         "cores": min(cores, shape.B * shape.H), "kind": "oracle",
-                         "sample": sample},
+        "data": "synthetic", "config": workload_config(args.config, args.gpus),
+        "cpu_baseline": {"value": rate, "unit": "tokens/s", "cores": used, "threads": cores,
+                         "kind": "oracle", "sample": sample},
         "e2e": {"value": rate, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def gla_sets(shape, dtype, dev, rank):
+    """Device buffer sets of one workload, enough of them that consecutive
+    steps never find their inputs in L2."""
+    import torch
+
+    q0, k0, v0, la0 = make_inputs(shape, dtype, seed=replica_seed(0, rank))
+    in_bytes = sum(t.numel() * t.element_size() for t in (q0, k0, v0, la0))
+    out_bytes = shape.B * shape.H * shape.tokens * shape.d_v * ESIZE[dtype]
+    set_bytes = in_bytes + len(DIRECTIONS) * out_bytes
+    R = max(2, math.ceil(2 * L2_BYTES / set_bytes))
+    sets = []
+    for _ in range(R):
+        ins = [t.to(dev) for t in (q0, k0, v0, la0)]
+        outs = [torch.empty((shape.B, shape.H, shape.grid_h, shape.grid_w, shape.d_v),
+                            dtype=q0.dtype, device=dev) for _ in DIRECTIONS]
+        fss = [torch.empty((shape.B, shape.H, shape.d_k, shape.d_v), dtype=torch.float32,
+                           device=dev) for _ in DIRECTIONS]
+        sets.append((ins, outs, fss))
+    return (q0, k0, v0, la0), sets, in_bytes, out_bytes
+
+
+def time_gla(name, K, W, dev, stream, rank, use_graph=True, chunk=64, with_eager=True):
+    """Time K steps (the four directions, one call each) of workload `name`
+    after W warm-up steps: the whole timed region and every call, with CUDA
+    events on the launching stream.  Returns the measurements as a dict."""
+    import torch
+    from recurrent_vision_backbone_chunkwise_b200 import gla
+
+    shape, dtype = CONFIGS[name]
+    host, sets, in_bytes, out_bytes = gla_sets(shape, dtype, dev, rank)
+    R = len(sets)
+    ws = torch.zeros(max(1, gla.gtr_gla_workspace_size(shape.B, shape.H, shape.grid_h,
+                                                         shape.grid_w, shape.d_k, shape.d_v,
+                                                         gla._DTYPE_CODE[host[0].dtype], chunk)),
+                     dtype=torch.uint8, device=dev)
+
+    def step(i, ev=None):
+        (q, k, v, la), outs, fss = sets[i % R]
+        for j, d in enumerate(DIRECTIONS):
+            if ev is not None:
+                ev[2 * j].record(stream)
+            gla.gtr_gla_fwd_ex(q, k, v, la, d, chunk=chunk, workspace=ws, out=outs[j],
+                               final_state=fss[j], stream=stream)
+            if ev is not None:
+                ev[2 * j + 1].record(stream)
+
+    with torch.cuda.stream(stream):
+        for i in range(W):
+            step(i)
+    stream.synchronize()
+    assert gla.gtr_gla_status(stream) == 0
+    call_events = [[torch.cuda.Event(enable_timing=True, external=use_graph) for _ in range(8)]
+                   for _ in range(K)]
+    graph = None
+    launches0 = gla.gtr_gla_launch_count()
+    if use_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for i in range(K):
+                step(i, call_events[i])
+        launches = gla.gtr_gla_launch_count() - launches0
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t0 = time.time()
+    launches_before = gla.gtr_gla_launch_count()
+    with torch.cuda.stream(stream):  # the graph replays on the current stream
+        start.record(stream)
+        if use_graph:
+            graph.replay()
+        else:
+            for i in range(K):
+                step(i, call_events[i])
+        end.record(stream)
+    torch.cuda.synchronize()
+    t1 = time.time()
+    if not use_graph:
+        launches = gla.gtr_gla_launch_count() - launches_before
+    assert gla.gtr_gla_status(stream) == 0
+    call_ms = [call_events[i][2 * j].elapsed_time(call_events[i][2 * j + 1])
+               for i in range(K) for j in range(len(DIRECTIONS))]
+    res = {"elapsed_ms": start.elapsed_time(end), "call_ms": call_ms, "eager_ms": call_ms,
+           "launches": int(launches), "wall": (t0, t1), "host": host, "sets": sets, "ws": ws,
+           "in_bytes": in_bytes, "out_bytes": out_bytes, "R": R, "step": step}
+    if graph is not None:
+        del graph
+        if with_eager:  # the same calls without graph capture (not the headline)
+            Ke = min(K, 200)
+            ev = [[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(Ke)]
+            with torch.cuda.stream(stream):
+                for i in range(Ke):
+                    step(i, ev[i])
+            stream.synchronize()
+            res["eager_ms"] = [ev[i][2 * j].elapsed_time(ev[i][2 * j + 1])
+                               for i in range(Ke) for j in range(len(DIRECTIONS))]
+    return res
+
+
+def roofline_entry(name, call_ms, chunk=64):
+    """The HBM roofline object of one workload from its per-call times."""
+    shape, dtype = CONFIGS[name]
+    call_bytes = workload_bytes(shape, dtype)
+    mean_s = statistics.mean(call_ms) / 1000.0
+    peak, peak_kind = measured_peaks()
+    achieved = call_bytes / mean_s / 1e9
+    return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak,
+            "traffic": profiled_traffic(name) if chunk == 64 else None,
+            "frac_vs_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
+            "peak_source": f"{peak_kind} copy bandwidth (burst)",
+            "bytes_per_call": call_bytes,
+            "timed_unit": "one library call (all kernels of one direction)"}
+
+
+def us_entry(call_ms, eager_ms):
+    return {"mean": 1e3 * statistics.mean(call_ms), "median": 1e3 * statistics.median(call_ms),
+            "min": 1e3 * min(call_ms), "eager_median": 1e3 * statistics.median(eager_ms),
+            "eager_min": 1e3 * min(eager_ms)}
+
+
+# The metric is quoted at 1600, 4096 and 16384 tokens: the default run times
+# these workloads too, after the headline one, and reports them under
+# "per_config" (same K and W, same timing method).
+PER_CONFIG = ("1024_b4", "16k_d64", "16k_d128")
 
 
 def main():
@@ -531,8 +696,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default="640_b1", choices=sorted(CONFIGS))
+    ap.add_argument("--chunk", type=int, default=64, choices=[32, 64, 128])
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="time only --config (skip the other token counts of the metric)")
     ap.add_argument("--op", default="gla", choices=["gla", "swiglu", "tail"],
                     help="gla: the headline (chunkwise GLA); swiglu: the Spatial SwiGLU block; "
                          "tail: the attention's output tail")
@@ -563,108 +731,37 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=180), device_id=dev)
 
     shape, dtype = CONFIGS[args.config]
-    q0, k0, v0, la0 = make_inputs(shape, dtype, seed=replica_seed(0, rank))
-    call_bytes = workload_bytes(shape, dtype)
-    in_bytes = sum(t.numel() * t.element_size() for t in (q0, k0, v0, la0))
-    out_bytes = shape.B * shape.H * shape.tokens * shape.d_v * ESIZE[dtype]
-    set_bytes = in_bytes + len(DIRECTIONS) * out_bytes
-    R = max(2, math.ceil(2 * L2_BYTES / set_bytes))
-    sets = []
-    for _ in range(R):
-        ins = [t.to(dev) for t in (q0, k0, v0, la0)]
-        outs = [torch.empty((shape.B, shape.H, shape.grid_h, shape.grid_w, shape.d_v),
-                            dtype=q0.dtype, device=dev) for _ in DIRECTIONS]
-        fss = [torch.empty((shape.B, shape.H, shape.d_k, shape.d_v), dtype=torch.float32,
-                           device=dev) for _ in DIRECTIONS]
-        sets.append((ins, outs, fss))
-    chunk = 64
-    ws = torch.zeros(max(1, gla.gtr_gla_workspace_size(shape.B, shape.H, shape.grid_h,
-                                                         shape.grid_w, shape.d_k, shape.d_v,
-                                                         gla._DTYPE_CODE[q0.dtype], chunk)),
-                     dtype=torch.uint8, device=dev)
-
+    chunk = args.chunk
     stream = torch.cuda.Stream(device=dev)
-
-    def step(i, ev=None):
-        (q, k, v, la), outs, fss = sets[i % R]
-        for j, d in enumerate(DIRECTIONS):
-            if ev is not None:
-                ev[2 * j].record(stream)
-            gla.gtr_gla_fwd_ex(q, k, v, la, d, chunk=chunk, workspace=ws, out=outs[j],
-                               final_state=fss[j], stream=stream)
-            if ev is not None:
-                ev[2 * j + 1].record(stream)
-
-    with torch.cuda.stream(stream):
-        for i in range(args.warmup):
-            step(i)
-    stream.synchronize()
-    assert gla.gtr_gla_status(stream) == 0
-
     use_graph = not args.no_graph
     K = args.steps
-    call_events = [[torch.cuda.Event(enable_timing=True, external=use_graph) for _ in range(8)]
-                   for _ in range(K)]
-    graph = None
-    launches0 = gla.gtr_gla_launch_count()
-    if use_graph:
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph, stream=stream):
-            for i in range(K):
-                step(i, call_events[i])
-        launches_per_replay = gla.gtr_gla_launch_count() - launches0
 
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
+    # warm-up and graph capture happen inside time_gla; the clock sampler runs
+    # from before the timed region to after it
     sampler = ClockSampler(smi_index(local))
     sampler.start()
     time.sleep(0.2)
     if world > 1:
         dist.barrier()
-    torch.cuda.synchronize()
-    t_wall0 = time.time()
-    launches_before = gla.gtr_gla_launch_count()
-    with torch.cuda.stream(stream):  # the graph replays on the current stream
-        start.record(stream)
-        if use_graph:
-            graph.replay()
-        else:
-            for i in range(K):
-                step(i, call_events[i])
-        end.record(stream)
-    torch.cuda.synchronize()
-    t_wall1 = time.time()
+    res = time_gla(args.config, K, args.warmup, dev, stream, rank, use_graph, chunk)
     if world > 1:
         dist.barrier()
-    gpu_launches = (launches_per_replay if use_graph
-                    else gla.gtr_gla_launch_count() - launches_before)
-    clocks = sampler.stop(t_wall0, t_wall1)
-    assert gla.gtr_gla_status(stream) == 0
+    clocks = sampler.stop(*res["wall"])
+    elapsed_ms = max_over_ranks(res["elapsed_ms"], device=dev)
+    call_ms, eager_ms = res["call_ms"], res["eager_ms"]
 
-    elapsed_ms = start.elapsed_time(end)
-    call_ms = [call_events[i][2 * j].elapsed_time(call_events[i][2 * j + 1])
-               for i in range(K) for j in range(len(DIRECTIONS))]
-    elapsed_ms = max_over_ranks(elapsed_ms, device=dev)
-    if graph is not None:
-        del graph
-
-    # the same calls without graph capture, for comparison (not the headline)
-    eager_ms = call_ms
-    if use_graph:
-        K_eager = min(K, 200)
-        ev_eager = [[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(K_eager)]
-        with torch.cuda.stream(stream):
-            for i in range(K_eager):
-                step(i, ev_eager[i])
-        stream.synchronize()
-        eager_ms = [ev_eager[i][2 * j].elapsed_time(ev_eager[i][2 * j + 1])
-                    for i in range(K_eager) for j in range(len(DIRECTIONS))]
-
-    # end-to-end through the public API with pinned host buffers
+    # end-to-end through the public API: inputs copied in from pinned host
+    # memory and every output and final state copied back, each step
+    sets, R, step = res["sets"], res["R"], res["step"]
+    q0, k0, v0, la0 = res["host"]
+    in_bytes, out_bytes = res["in_bytes"], res["out_bytes"]
+    fs_bytes = shape.B * shape.H * shape.d_k * shape.d_v * 4
     K_e2e = min(K, 200)
     host_in = [t.pin_memory() for t in (q0, k0, v0, la0)]
     host_out = [torch.empty(sets[0][1][0].shape, dtype=q0.dtype).pin_memory()
                 for _ in DIRECTIONS]
+    host_fs = [torch.empty(sets[0][2][0].shape, dtype=torch.float32).pin_memory()
+               for _ in DIRECTIONS]
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
@@ -679,54 +776,73 @@ def main():
             for dst, src in zip((q, k, v, la), host_in):
                 dst.copy_(src, non_blocking=True)
             for j, d in enumerate(DIRECTIONS):
-                gla.gtr_gla_fwd(q, k, v, la, d, out=outs[j], final_state=fss[j], stream=stream)
+                if chunk == 64 and dtype == "f16":
+                    gla.gtr_gla_fwd(q, k, v, la, d, out=outs[j], final_state=fss[j], stream=stream)
+                else:
+                    gla.gtr_gla_fwd_ex(q, k, v, la, d, chunk=chunk, workspace=res["ws"],
+                                       out=outs[j], final_state=fss[j], stream=stream)
                 host_out[j].copy_(outs[j], non_blocking=True)
+                host_fs[j].copy_(fss[j], non_blocking=True)
         e1.record(stream)
     stream.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    e2e_ms = max_over_ranks(e2e_ms, device=dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), device=dev)
 
-    tokens_per_step = len(DIRECTIONS) * shape.B * shape.H * shape.tokens
+    tokens_per_step = len(DIRECTIONS) * image_tokens(shape)
     value = aggregate_rate(world, K, tokens_per_step, elapsed_ms)
     e2e_value = aggregate_rate(world, K_e2e, tokens_per_step, e2e_ms)
-    mean_call_s = statistics.mean(call_ms) / 1000.0
-    peak, peak_kind = measured_peaks()
-    achieved = call_bytes / mean_call_s / 1e9
-
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": elapsed_ms / K, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": dtype, "data": "synthetic",
-        "config": {"workload": args.config, "B": shape.B, "H": shape.H,
-                   "grid": [shape.grid_h, shape.grid_w], "tokens": shape.tokens,
-                   "d_k": shape.d_k, "d_v": shape.d_v, "chunk": chunk, "directions": 4,
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": f"inputs rotate over {R} buffer sets "
-                         f"({R * set_bytes / 2**20:.0f} MiB > 126 MiB L2)",
-                   "cuda_graph": use_graph},
-        "kernel_us_per_call": {"mean": 1e6 * mean_call_s,
-                               "median": 1e3 * statistics.median(call_ms),
-                               "min": 1e3 * min(call_ms),
-                               "eager_median": 1e3 * statistics.median(eager_ms),
-                               "eager_min": 1e3 * min(eager_ms)},
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": profiled_traffic(args.config),
-                     "frac_vs_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
-                     "peak_source": f"{peak_kind} copy bandwidth",
-                     "bytes_per_call": call_bytes,
-                     "timed_unit": "one library call (all kernels of one direction)"},
-        "gpu_launches": int(gpu_launches),
+        "config": workload_config(args.config, world, chunk),
+        "timing": {"cuda_graph": use_graph, "per_call": "CUDA events around every call"},
+        "kernel_us_per_call": us_entry(call_ms, eager_ms),
+        "token_heads_per_s": value * shape.H,
+        "roofline": roofline_entry(args.config, call_ms, chunk),
+        "gpu_launches": res["launches"],
         "e2e": {"value": e2e_value, "unit": "tokens/s",
                 "h2d_bytes_per_step": in_bytes,
-                "d2h_bytes_per_step": len(DIRECTIONS) * out_bytes, "steps": K_e2e},
+                "d2h_bytes_per_step": len(DIRECTIONS) * (out_bytes + fs_bytes), "steps": K_e2e},
         "clocks": clocks,
     }
+    del res, sets, step
+    torch.cuda.empty_cache()
+
+    if not args.no_per_config and chunk == 64:
+        per = {}
+        for name in PER_CONFIG:
+            if name == args.config:
+                continue
+            sampler = ClockSampler(smi_index(local))
+            sampler.start()
+            time.sleep(0.2)
+            if world > 1:
+                dist.barrier()
+            r = time_gla(name, K, args.warmup, dev, stream, rank, use_graph, chunk)
+            if world > 1:
+                dist.barrier()
+            ck = sampler.stop(*r["wall"])
+            el = max_over_ranks(r["elapsed_ms"], device=dev)
+            s2, _ = CONFIGS[name]
+            per[name] = {"tokens": s2.tokens, "config": workload_config(name, world, chunk),
+                         "value": aggregate_rate(world, K, len(DIRECTIONS) * image_tokens(s2), el),
+                         "unit": "tokens/s", "ms_per_step": el / K,
+                         "kernel_us_per_call": us_entry(r["call_ms"], r["eager_ms"]),
+                         "roofline": roofline_entry(name, r["call_ms"], chunk),
+                         "gpu_launches": r["launches"], "clocks": ck}
+            del r
+            torch.cuda.empty_cache()
+        line["per_config"] = per
+
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, cores, reps, el = cpu_oracle_rate(shape, dtype, seconds=10.0)
-        line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": cores,
-                                "kind": "oracle",
-                                "sample": f"{reps} steps x 4 directions of the full "
-                                          f"workload in {el:.1f} s"}
+        base = cpu_oracle_rate(shape, dtype, seconds=10.0)
+        base["single_thread"] = cpu_oracle_rate(shape, dtype, seconds=4.0, threads=1)
+        line["cpu_baseline"] = base
+        for name, entry in line.get("per_config", {}).items():
+            s2, d2 = CONFIGS[name]
+            b2 = cpu_oracle_rate(s2, d2, seconds=3.0)
+            b2["single_thread"] = cpu_oracle_rate(s2, d2, seconds=1.5, threads=1)
+            entry["cpu_baseline"] = b2
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -93,6 +93,35 @@ def _shape(q, v):
     return B, H, gh, gw, dk, v.shape[-1]
 
 
+def _check(name, t, shape, dtype, device):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype} (got {t.dtype})")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)} (got {tuple(t.shape)})")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.device.type != "cuda" or t.device != device:
+        raise ValueError(f"{name} must be on the CUDA device of q (got {t.device})")
+
+
+def _validate(q, k, v, log_alpha, out, final_state):
+    """Host-side checks before any call: the library reads and writes the
+    tensors through raw pointers, so a wrong shape, dtype, layout or device
+    would make it touch memory outside them."""
+    B, H, gh, gw, dk, dv = _shape(q, v)
+    dev = q.device
+    _check("q", q, (B, H, gh, gw, dk), q.dtype, dev)
+    _check("k", k, (B, H, gh, gw, dk), q.dtype, dev)
+    _check("v", v, (B, H, gh, gw, dv), q.dtype, dev)
+    _check("log_alpha", log_alpha, (B, H, gh, gw, dk), torch.float32, dev)
+    if out is not None:
+        _check("out", out, (B, H, gh, gw, dv), q.dtype, dev)
+    if final_state is not None:
+        _check("final_state", final_state, (B, H, dk, dv), torch.float32, dev)
+
+
 def _alloc_out(q, v, out, final_state, want_state):
     B, H, gh, gw, dk, dv = _shape(q, v)
     if out is None:
@@ -107,6 +136,7 @@ def gtr_gla_fwd(q, k, v, log_alpha, direction, out=None, final_state=None,
     """fp16 forward, chunk 64, library-owned workspace.  Returns (out, final_state)."""
     if q.dtype != torch.float16 or k.dtype != torch.float16 or v.dtype != torch.float16:
         raise ValueError("gtr_gla_fwd takes fp16 q, k, v (use gtr_gla_fwd_ex for others)")
+    _validate(q, k, v, log_alpha, out, final_state)
     out, final_state = _alloc_out(q, v, out, final_state, want_state)
     B, H, gh, gw, dk, dv = _shape(q, v)
     rc = _lib.gtr_gla_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(out),
@@ -121,12 +151,15 @@ def gtr_gla_fwd_ex(q, k, v, log_alpha, direction, chunk=64, workspace=None, out=
                    final_state=None, want_state=True, stream=None):
     """Forward with the dtype taken from q and a caller workspace (allocated here
     as a zero-filled uint8 CUDA tensor if not given).  Returns (out, final_state)."""
+    _validate(q, k, v, log_alpha, out, final_state)
     out, final_state = _alloc_out(q, v, out, final_state, want_state)
     B, H, gh, gw, dk, dv = _shape(q, v)
     dtype = _DTYPE_CODE.get(q.dtype)
     if dtype is None:
         raise ValueError(f"unsupported dtype {q.dtype}")
     need = gtr_gla_workspace_size(B, H, gh, gw, dk, dv, dtype, chunk)
+    if workspace is not None and (workspace.device != q.device or not workspace.is_contiguous()):
+        raise ValueError("workspace must be a contiguous tensor on q's device")
     if workspace is None and need > 0:
         workspace = torch.zeros(need, dtype=torch.uint8, device=q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
@@ -145,6 +178,9 @@ def gtr_gla_fwd_noalloc(q, k, v, log_alpha, direction, out, final_state=None, st
     array.  Returns (out, final_state)."""
     if q.dtype != torch.float16 or k.dtype != torch.float16 or v.dtype != torch.float16:
         raise ValueError("gtr_gla_fwd_noalloc takes fp16 q, k, v")
+    if out is None:
+        raise ValueError("gtr_gla_fwd_noalloc needs a caller-given out")
+    _validate(q, k, v, log_alpha, out, final_state)
     B, H, gh, gw, dk, dv = _shape(q, v)
     rc = _lib.gtr_gla_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(out),
                                   _ptr(final_state), B, H, gh, gw, dk, dv, int(direction),

@@ -164,3 +164,47 @@ def test_output_tail_argument_errors_before_launch(gla):
     assert call(dtype=gla.F32) == -6
     assert call(ptrs=q[:2] + [C.c_void_p((1 << 20) + (2 << 32) + 8), q[3]]) == -5   # w misaligned
     assert call(ptrs=q[:3] + [q[0]]) == -11              # y is o
+
+
+def _tensors(dt=None):
+    import torch
+
+    dt = dt or torch.float16
+    q = torch.zeros((1, 2, 4, 5, 64), dtype=dt)
+    return q, q.clone(), torch.zeros((1, 2, 4, 5, 64), dtype=dt), torch.zeros((1, 2, 4, 5, 64))
+
+
+@pytest.mark.parametrize("bad", ["la_f16", "k_shape", "v_dtype", "out_small", "out_strided",
+                                 "fs_f16", "fs_shape", "cpu"])
+def test_binding_checks_tensors_before_any_call(gla, bad):
+    """The binding rejects tensors whose dtype, shape, layout or device would
+    make the library read or write outside them, before calling it (these
+    checks need no GPU: every tensor here is a CPU tensor, and the device is
+    checked last)."""
+    import torch
+
+    q, k, v, la = _tensors()
+    out, fs = None, None
+    if bad == "la_f16":
+        la = la.half()
+    elif bad == "k_shape":
+        k = k[..., :32].contiguous()
+    elif bad == "v_dtype":
+        v = v.bfloat16()
+    elif bad == "out_small":
+        out = torch.zeros((1, 2, 4, 4, 64), dtype=torch.float16)
+    elif bad == "out_strided":
+        out = torch.zeros((1, 2, 4, 5, 128), dtype=torch.float16)[..., ::2]
+    elif bad == "fs_f16":
+        fs = torch.zeros((1, 2, 64, 64), dtype=torch.float16)
+    elif bad == "fs_shape":
+        fs = torch.zeros((1, 2, 64, 32))
+    before = gla.gtr_gla_launch_count()
+    for fn in (gla.gtr_gla_fwd, gla.gtr_gla_fwd_ex):
+        with pytest.raises(ValueError) as e:
+            fn(q, k, v, la, 0, out=out, final_state=fs)
+        if bad == "cpu":
+            assert "CUDA device" in str(e.value)
+    with pytest.raises(ValueError):
+        gla.gtr_gla_fwd_noalloc(q, k, v, la, 0, out if out is not None else torch.zeros_like(v), fs)
+    assert gla.gtr_gla_launch_count() == before

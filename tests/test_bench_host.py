@@ -108,3 +108,23 @@ def test_nvidia_smi_index_and_single_rank_group(monkeypatch):
 
     assert bench.dist_setup(One(), None) is None
     bench.dist_barrier(None)  # a no-op without a group
+
+
+def test_tokens_per_call_are_image_tokens():
+    """tokens/s counts image tokens, B * grid_h * grid_w per call: every head
+    of a token is processed by the same call and is not counted again."""
+    from recurrent_vision_backbone_chunkwise_b200.inputs import CONFIGS
+
+    assert bench.image_tokens(CONFIGS["640_b1"][0]) == 1600
+    assert bench.image_tokens(CONFIGS["1024_b4"][0]) == 4 * 4096
+    assert bench.image_tokens(CONFIGS["16k_d128"][0]) == 16384
+
+
+def test_both_arms_print_the_same_config():
+    """The reference arm and the GPU arm describe a workload with one function,
+    so their config objects are equal for every workload and world size."""
+    for name in ("640_b1", "1024_b4", "16k_d64", "16k_d128"):
+        for world in (1, 2):
+            a, b = bench.workload_config(name, world), bench.workload_config(name, world)
+            assert a == b and a["workload"] == name and a["tokens"] > 0
+    assert set(bench.PER_CONFIG) == {"1024_b4", "16k_d64", "16k_d128"}
