@@ -460,6 +460,19 @@ def image_tokens(shape) -> int:
     return shape.B * shape.tokens
 
 
+_HOST_THREADS = []
+
+
+def host_threads() -> int:
+    """OpenMP threads of the host (all cores), read once: a call with an
+    explicit thread count changes what OpenMP reports afterwards."""
+    if not _HOST_THREADS:
+        import oracle
+
+        _HOST_THREADS.append(int(oracle.max_threads()))
+    return _HOST_THREADS[0]
+
+
 def oracle_sample(shape, dtype, seconds: float):
     """Inputs of a bounded CPU sample of `shape`: the grid is cut to its first
     rows so that one direction of every plane takes about `seconds` / 4 on
@@ -469,7 +482,7 @@ def oracle_sample(shape, dtype, seconds: float):
     import oracle
 
     q, k, v, la = (t.double().numpy() for t in make_inputs(shape, dtype, seed=0))
-    cores = oracle.max_threads()
+    cores = host_threads()
     rows = shape.grid_h
     probe = max(1, min(rows, 8))
     t0 = time.perf_counter()
@@ -489,7 +502,7 @@ def cpu_oracle_rate(shape, dtype, seconds: float = 10.0, threads=None, max_reps:
     import oracle
 
     (q, k, v, la), rows = oracle_sample(shape, dtype, seconds if threads != 1 else seconds / 8)
-    cores = oracle.max_threads() if threads is None else int(threads)
+    cores = host_threads() if threads is None else int(threads)
     used = min(cores, shape.B * shape.H)
     reps = 0
     t0 = time.perf_counter()
@@ -536,7 +549,7 @@ def run_reference(args):
     shape, dtype = CONFIGS[args.config]
     budget = 60.0 / (args.steps + args.warmup)  # seconds of host time per step
     (qs, ks, vs, las), rows = oracle_sample(shape, dtype, 4.0 * budget)
-    cores = oracle.max_threads()
+    cores = host_threads()
     for i in range(args.warmup):
         oracle.forward(qs, ks, vs, las, DIRECTIONS[i % 4], n_threads=cores)
     t0 = time.perf_counter()

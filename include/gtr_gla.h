@@ -79,7 +79,11 @@ enum {
                                          was not zero-filled); reported by
                                          gtr_gla_status, the call did no work in the
                                          affected segments and the header is clean
-                                         again afterwards                          */
+                                         again afterwards                          */,
+    GTR_GLA_ERR_RANGE = -13       /* fp16 I/O only, reported by gtr_gla_status: the
+                                     fp16 copy of a carried state, the tensor-core
+                                     operand of q S, exceeded 65504 in magnitude;
+                                     the output is written but not exact           */
 };
 
 /* ---- entry points --------------------------------------------------- */

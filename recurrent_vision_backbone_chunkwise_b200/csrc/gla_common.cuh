@@ -41,7 +41,7 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 }
 
 // Device-side error codes latched into the library's error word.
-enum : int { kDevErrNone = 0, kDevErrTimeout = 1, kDevErrWorkspace = 2 };
+enum : int { kDevErrNone = 0, kDevErrTimeout = 1, kDevErrWorkspace = 2, kDevErrRange = 3 };
 
 __device__ __forceinline__ void latch_error(int *err, int code) {
     if (err) atomicCAS(err, 0, code);

@@ -223,6 +223,7 @@ int gtr_gla_status(cudaStream_t stream) {
         return GTR_GLA_ERR_CUDA;
     if (host_err == kDevErrTimeout) return GTR_GLA_ERR_TIMEOUT;
     if (host_err == kDevErrWorkspace) return GTR_GLA_ERR_WORKSPACE_STATE;
+    if (host_err == kDevErrRange) return GTR_GLA_ERR_RANGE;
     return host_err ? GTR_GLA_ERR_CUDA : GTR_GLA_OK;
 }
 
@@ -242,6 +243,8 @@ const char *gtr_gla_strerror(int code) {
         case GTR_GLA_ERR_ALIAS: return "output overlaps an input";
         case GTR_GLA_ERR_WORKSPACE_STATE:
             return "workspace header not zero when a call started (overlapping calls sharing it?)";
+        case GTR_GLA_ERR_RANGE:
+            return "a carried state exceeded the fp16 operand range (the output is not exact)";
         default: return "unknown error code";
     }
 }
