@@ -80,6 +80,10 @@ def test_tail_traffic_follows_its_own_code_hash(tmp_path, monkeypatch):
     prof = "output_tail_kernel_1024_b4.md"
     shutil.copy(os.path.join(ROOT, "profiles", prof), tmp_path / "profiles")
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    # the copy names the current code's hash, as a fresh capture would
+    _edit(tmp_path / "profiles" / prof,
+          lambda t: "kernel_code_sha256_16: %s\n" % bench.kernel_code_hash(bench.TAIL_FILES) +
+          t.replace("kernel_code_sha256_16", "earlier_hash"))
     got = bench.profiled_traffic("1024_b4", prof, bench.TAIL_FILES)
     assert isinstance(got, int) and got > 0
     _edit(tmp_path / CSRC / "gla_fused.cu", lambda t: t + "\nconstexpr int kProbe = 3;\n")
