@@ -267,6 +267,124 @@ def run_swiglu(args):
         dist.destroy_process_group()
 
 
+def run_backbone(args):
+    """Backbone leg (not the headline): the 12-layer stack (direction = layer
+    mod 4) on the workload's grid and batch, width C = 64 H and F = 4 C, all
+    12 layers in one CUDA graph per step; images/s and the latency of one
+    forward, the fp64 oracle's layers on the host as the CPU baseline."""
+    import torch
+    from recurrent_vision_backbone_chunkwise_b200 import gla, layer
+    from recurrent_vision_backbone_chunkwise_b200.inputs import make_backbone_params
+
+    ri = rank_info()
+    torch.cuda.set_device(ri.local_rank)
+    dev = torch.device("cuda", ri.local_rank)
+    dist = dist_setup(ri, dev)
+    shape, _ = CONFIGS[args.config]
+    B, gh, gw, C = shape.B, shape.grid_h, shape.grid_w, 64 * shape.H
+    F, n_layers = 4 * C, 12
+    params = make_backbone_params(C, F, n_layers, "f16", seed=replica_seed(0, ri.rank))
+    w_bytes = sum(t.numel() * t.element_size() for p in params for t in p.values())
+    # weight sets rotate so that the weights a step reads exceed L2
+    R = max(1, math.ceil(L2_BYTES / w_bytes) + (1 if w_bytes < L2_BYTES else 0))
+    wsets = [[layer.pack_weights(p, dev) for p in params] for _ in range(R)]
+    g = torch.Generator().manual_seed(replica_seed(1, ri.rank))
+    x0 = torch.randn(B, gh, gw, C, generator=g).half()
+    xs = [x0.to(dev) for _ in range(R)]
+    ws = torch.zeros(layer.gtr_layer_workspace_size(B, gh, gw, C, F), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(i, ev=None):
+        x = xs[i % R]
+        if ev is not None:
+            ev[0].record(stream)
+        layer.gtr_backbone_fwd(x, wsets[i % R], workspace=ws, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            step(i)
+    stream.synchronize()
+    assert gla.gtr_gla_status(stream) == 0
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)] for _ in range(K)]
+    launches0 = gla.gtr_gla_launch_count()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(K):
+            step(i, evs[i])
+    launches = gla.gtr_gla_launch_count() - launches0
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(smi_index(ri.local_rank))
+    sampler.start()
+    time.sleep(0.2)
+    dist_barrier(dist)
+    torch.cuda.synchronize()
+    t0 = time.time()
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        graph.replay()
+        end.record(stream)
+    torch.cuda.synchronize()
+    t1 = time.time()
+    dist_barrier(dist)
+    clocks = sampler.stop(t0, t1)
+    assert gla.gtr_gla_status(stream) == 0
+    elapsed = max_over_ranks(start.elapsed_time(end), device=dev)
+    call_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    del graph
+    # end to end: the image's tokens in from pinned host memory, the features
+    # back, every step, through the public entry point
+    hx = x0.pin_memory()
+    hy = torch.empty_like(x0).pin_memory()
+    K2 = min(K, 100)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist_barrier(dist)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(K2):
+            x = xs[i % R]
+            x.copy_(hx, non_blocking=True)
+            layer.gtr_backbone_fwd(x, wsets[i % R], workspace=ws, stream=stream)
+            hy.copy_(x, non_blocking=True)
+        e1.record(stream)
+    stream.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), device=dev)
+    line = {
+        "metric": "GTR backbone (12 layers) images/s and ms per forward", "value":
+            aggregate_rate(ri.world, K, B, elapsed), "unit": "images/s", "n_gpus": ri.world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": elapsed / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "config": {"workload": f"backbone_{args.config}", "B": B, "grid": [gh, gw], "C": C, "F": F,
+                   "layers": n_layers, "heads": C // 64,
+                   "l2": f"weights rotate over {R} sets ({R * w_bytes / 2**20:.0f} MiB > 126 MiB L2)",
+                   "cuda_graph": True},
+        "ms_per_forward": {"mean": statistics.mean(call_ms), "median": statistics.median(call_ms),
+                           "min": min(call_ms)},
+        "gpu_launches": int(launches),
+        "e2e": {"value": aggregate_rate(ri.world, K2, B, e2e_ms), "unit": "images/s",
+                "h2d_bytes_per_step": x0.numel() * 2, "d2h_bytes_per_step": x0.numel() * 2, "steps": K2},
+        "clocks": clocks,
+    }
+    if ri.rank == 0 and ri.world == 1 and not args.no_cpu_baseline:
+        import oracle.backbone as obb
+
+        reps, t0 = 0, time.perf_counter()
+        x = x0
+        while time.perf_counter() - t0 < 10.0 and reps < n_layers:
+            x = obb.layer_forward(x, params[reps], reps % 4)
+            reps += 1
+        el = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": B * reps / n_layers / el, "unit": "images/s", "cores": host_threads(),
+                                "kind": "oracle",
+                                "sample": f"{reps} of the {n_layers} layers (fp64) in {el:.1f} s"}
+    if ri.rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
 def run_tail(args):
     """Output-tail leg (not the headline): token-heads/s of the tail on the
     workload's attention output (B, H, grid, d_v), its HBM roofline fraction
@@ -714,9 +832,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-config", action="store_true",
                     help="time only --config (skip the other token counts of the metric)")
-    ap.add_argument("--op", default="gla", choices=["gla", "swiglu", "tail"],
+    ap.add_argument("--op", default="gla", choices=["gla", "swiglu", "tail", "backbone"],
                     help="gla: the headline (chunkwise GLA); swiglu: the Spatial SwiGLU block; "
-                         "tail: the attention's output tail")
+                         "tail: the attention's output tail; backbone: the 12-layer stack")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.op == "swiglu" and args.impl == "ours":
@@ -724,6 +842,9 @@ def main():
         return
     if args.op == "tail" and args.impl == "ours":
         run_tail(args)
+        return
+    if args.op == "backbone" and args.impl == "ours":
+        run_backbone(args)
         return
 
     if args.impl == "reference":

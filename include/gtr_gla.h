@@ -80,10 +80,9 @@ enum {
                                          gtr_gla_status, the call did no work in the
                                          affected segments and the header is clean
                                          again afterwards                          */,
-    GTR_GLA_ERR_RANGE = -13       /* fp16 I/O only, reported by gtr_gla_status: the
-                                     fp16 copy of a carried state, the tensor-core
-                                     operand of q S, exceeded 65504 in magnitude;
-                                     the output is written but not exact           */
+    GTR_GLA_ERR_BOUNDS = -13      /* checked build (libgtr_gla_checked.so) only,
+                                     reported by gtr_gla_status: a kernel's index
+                                     check failed; that access was skipped       */
 };
 
 /* ---- entry points --------------------------------------------------- */
@@ -145,6 +144,38 @@ int gtr_gla_fwd_ex(const void *q, const void *k, const void *v, const float *log
 int gtr_gla_fwd_noalloc(const void *q, const void *k, const void *v, const float *log_alpha,
                         void *out, float *final_state, int B, int H, int grid_h, int grid_w,
                         int d_k, int d_v, int direction, cudaStream_t stream);
+
+/*
+ * gtr_gla_fwd_tail -- the forward pass followed by the output tail of GTR's
+ * token mixer, with the tail fused into the attention's output stores
+ * ("GTR: Gated Token Recurrence for Efficient Dense Prediction", x-techcon
+ * article, section 算子: the operator's benchmark leaves this fusion out; the
+ * pages do not define the tail, and the reading used is the per-token
+ * epilogue of gtr_output_tail.h):
+ *     y[b, r, h*d_v + j] = o[b, h, r, j] / sqrt(mean_j' o[b, h, r, j']^2 + eps)
+ *                          * w_n[h, j] * SiLU(z[b, r, h*d_v + j])
+ * with o the attention output of gtr_gla_fwd_ex (never written to memory when
+ * d_k = d_v = 64: the norm is taken on its fp32 value and y is rounded once).
+ *   z, y:      [B, grid_h, grid_w, H*d_v] in the I/O dtype (heads merged
+ *              channels-last); y must not overlap any input.
+ *   w_n:       [H, d_v] fp32.  eps: finite, >= 0.
+ *   dtype:     GTR_GLA_F16 or GTR_GLA_BF16 (chunk 64).
+ *   workspace: gtr_gla_tail_workspace_size(...) bytes, 256-byte aligned,
+ *              zero-filled before its first use (as for gtr_gla_fwd_ex).
+ *              Head sizes of 128 keep o there and run the tail as a second
+ *              launch (gtr_output_tail_fwd).
+ * Other arguments, errors and final_state as gtr_gla_fwd_ex; in addition
+ * GTR_GLA_ERR_NULL for a NULL z or w_n, _SHAPE for eps < 0 or not finite,
+ * _ALIGN for z or w_n, _ALIAS when y overlaps z, w_n or the workspace.
+ */
+int gtr_gla_fwd_tail(const void *q, const void *k, const void *v, const float *log_alpha,
+                     const void *z, const float *w_n, float eps, void *y, float *final_state,
+                     int B, int H, int grid_h, int grid_w, int d_k, int d_v, int direction,
+                     int dtype, void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Workspace bytes of gtr_gla_fwd_tail (0 for invalid sizes or dtypes). */
+size_t gtr_gla_tail_workspace_size(int B, int H, int grid_h, int grid_w, int d_k, int d_v,
+                                   int dtype);
 
 /* Workspace bytes gtr_gla_fwd_ex needs for this problem (0 if none). */
 size_t gtr_gla_workspace_size(int B, int H, int grid_h, int grid_w, int d_k, int d_v,

@@ -1,11 +1,17 @@
 """Build libgtr_gla.so in-tree with nvcc for sm_100a (no JIT, no torch extension).
 
-    python -m recurrent_vision_backbone_chunkwise_b200.build [--force] [--verbose]
+    python -m recurrent_vision_backbone_chunkwise_b200.build [--force] [--verbose] [--checked]
 
 Every ``csrc/*.cu`` is compiled to an object with
 ``-gencode arch=compute_100a,code=sm_100a -O3 -lineinfo`` and linked into one
 shared library with the CUDA runtime linked statically.  Objects are rebuilt
 only when a source or header is newer than them.
+
+``checked=True`` builds libgtr_gla_checked.so from the same sources with
+``-DGTR_CHECKED``: every computed global index and TMA coordinate of the
+kernels is checked before use, a failed check is latched as
+GTR_GLA_ERR_BOUNDS (read by gtr_gla_status) and the access is skipped.  It is
+the debugging stand-in for a memory checker, with the same entry points.
 """
 from __future__ import annotations
 
@@ -21,6 +27,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libgtr_gla.so")
+BUILD_CHECKED = os.path.join(PKG, "_build_checked")
+LIB_CHECKED = os.path.join(PKG, "libgtr_gla_checked.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 # cuBLASLt runs the dense projections of the Spatial SwiGLU block
@@ -43,15 +51,17 @@ def _newest_dep() -> float:
     return max(os.path.getmtime(d) for d in deps if os.path.exists(d))
 
 
-def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None,
+          checked: bool = False) -> str:
+    build_dir, lib = (BUILD_CHECKED, LIB_CHECKED) if checked else (BUILD, LIB)
+    os.makedirs(build_dir, exist_ok=True)
     nvcc = _nvcc()
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     dep_t = _newest_dep()
-    flags = NVFLAGS + (extra or [])
+    flags = NVFLAGS + (["-DGTR_CHECKED"] if checked else []) + (extra or [])
 
     def compile_one(src: str) -> str:
-        obj = os.path.join(BUILD, os.path.basename(src) + ".o")
+        obj = os.path.join(build_dir, os.path.basename(src) + ".o")
         if (not force and os.path.exists(obj)
                 and os.path.getmtime(obj) >= max(os.path.getmtime(src), dep_t)):
             return obj
@@ -69,14 +79,15 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
 
     with ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
         objs = list(ex.map(compile_one, srcs))
-    if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < max(os.path.getmtime(o) for o in objs):
-        cmd = [nvcc] + ARCH + ["-shared", "-cudart", "static", "-o", LIB + ".tmp"] + objs + LINK
+    if force or not os.path.exists(lib) or os.path.getmtime(lib) < max(os.path.getmtime(o) for o in objs):
+        cmd = [nvcc] + ARCH + ["-shared", "-cudart", "static", "-o", lib + ".tmp"] + objs + LINK
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-        os.replace(LIB + ".tmp", LIB)
-    return LIB
+        os.replace(lib + ".tmp", lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv,
+                checked="--checked" in sys.argv))

@@ -40,11 +40,33 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
     return __float2bfloat16_rn(x);
 }
 
+// SiLU(z) = z * sigmoid(z) = z/2 * (1 + tanh(z/2)): one hardware tanh (relative
+// error about 2^-11, that of an fp16 rounding of the result).
+__device__ __forceinline__ float silu_f32(float z) {
+    float t;
+    const float hz = 0.5f * z;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(hz));
+    return fmaf(hz, t, hz);
+}
+
 // Device-side error codes latched into the library's error word.
-enum : int { kDevErrNone = 0, kDevErrTimeout = 1, kDevErrWorkspace = 2, kDevErrRange = 3 };
+enum : int { kDevErrNone = 0, kDevErrTimeout = 1, kDevErrWorkspace = 2, kDevErrBounds = 3 };
 
 __device__ __forceinline__ void latch_error(int *err, int code) {
     if (err) atomicCAS(err, 0, code);
 }
+
+// Index checks of the checked build (-DGTR_CHECKED, libgtr_gla_checked.so):
+// every computed global index and TMA coordinate is tested before use; a
+// failed test latches kDevErrBounds and the caller skips the access.  In the
+// normal build the test compiles away.
+#ifdef GTR_CHECKED
+__device__ __forceinline__ bool index_ok(bool ok, int *err) {
+    if (!ok) latch_error(err, kDevErrBounds);
+    return ok;
+}
+#else
+__device__ __forceinline__ bool index_ok(bool, int *) { return true; }
+#endif
 
 }  // namespace gtr

@@ -25,7 +25,7 @@ template <typename T, int DK, int DV, int C>
 __global__ void __launch_bounds__(kGenThreads)
 gla_chunk_state_kernel(const T *__restrict__ k, const T *__restrict__ v,
                        const float *__restrict__ la, float *__restrict__ dS,
-                       float *__restrict__ gam, int n, int gh, int gw, int dir, int nc) {
+                       float *__restrict__ gam, int n, int gh, int gw, int dir, int nc, int *err) {
     extern __shared__ float sm[];
     float *b = sm;            // [C][DK]  log-gate prefix sums
     float *kh = b + C * DK;   // [C][DK]  k, then k . e^{g - b}
@@ -38,8 +38,8 @@ gla_chunk_state_kernel(const T *__restrict__ k, const T *__restrict__ v,
     for (int e = threadIdx.x; e < C * DK; e += blockDim.x) {
         const int u = e / DK, i = e % DK;
         float lv = 0.f, kv = 0.f;
-        if (u < len) {
-            const size_t r = (size_t)scan_to_raster(t0 + u, n, gh, gw, dir);
+        const size_t r = (size_t)scan_to_raster(t0 + u, n, gh, gw, dir);
+        if (u < len && index_ok(r < (size_t)n, err)) {
             lv = la[pk + r * DK + i];
             kv = to_f32(k[pk + r * DK + i]);
         }
@@ -49,10 +49,8 @@ gla_chunk_state_kernel(const T *__restrict__ k, const T *__restrict__ v,
     for (int e = threadIdx.x; e < C * DV; e += blockDim.x) {
         const int u = e / DV, j = e % DV;
         float vv = 0.f;
-        if (u < len) {
-            const size_t r = (size_t)scan_to_raster(t0 + u, n, gh, gw, dir);
-            vv = to_f32(v[pv + r * DV + j]);
-        }
+        const size_t r = (size_t)scan_to_raster(t0 + u, n, gh, gw, dir);
+        if (u < len && index_ok(r < (size_t)n, err)) vv = to_f32(v[pv + r * DV + j]);
         vs[e] = vv;
     }
     __syncthreads();
@@ -141,7 +139,7 @@ __global__ void __launch_bounds__(kGenThreads)
 gla_chunk_output_kernel(const T *__restrict__ q, const T *__restrict__ k,
                         const T *__restrict__ v, const float *__restrict__ la,
                         const float *__restrict__ Sin, T *__restrict__ o, int n, int gh,
-                        int gw, int dir, int nc) {
+                        int gw, int dir, int nc, int *err) {
     constexpr int DKP = DK + 1;  // padded rows: pair loops read one row per lane
     constexpr int CP = C + 1;
     extern __shared__ float sm[];
@@ -159,8 +157,8 @@ gla_chunk_output_kernel(const T *__restrict__ q, const T *__restrict__ k,
     for (int e = threadIdx.x; e < C * DK; e += blockDim.x) {
         const int u = e / DK, i = e % DK;
         float qv = 0.f, kv = 0.f, lv = 0.f;
-        if (u < len) {
-            const size_t r = (size_t)scan_to_raster(t0 + u, n, gh, gw, dir);
+        const size_t r = (size_t)scan_to_raster(t0 + u, n, gh, gw, dir);
+        if (u < len && index_ok(r < (size_t)n, err)) {
             qv = to_f32(q[pk + r * DK + i]);
             kv = to_f32(k[pk + r * DK + i]);
             lv = la[pk + r * DK + i];
@@ -172,10 +170,8 @@ gla_chunk_output_kernel(const T *__restrict__ q, const T *__restrict__ k,
     for (int e = threadIdx.x; e < C * VT; e += blockDim.x) {
         const int u = e / VT, j = e % VT;
         float vv = 0.f;
-        if (u < len) {
-            const size_t r = (size_t)scan_to_raster(t0 + u, n, gh, gw, dir);
-            vv = to_f32(v[pv + r * DV + j0 + j]);
-        }
+        const size_t r = (size_t)scan_to_raster(t0 + u, n, gh, gw, dir);
+        if (u < len && index_ok(r < (size_t)n, err)) vv = to_f32(v[pv + r * DV + j0 + j]);
         vs[e] = vv;
     }
     const float *Sg = Sin + ((size_t)bh * nc + c) * DK * DV;
@@ -244,6 +240,7 @@ gla_chunk_output_kernel(const T *__restrict__ q, const T *__restrict__ k,
         const int u = tt + 16 * a;
         if (u >= len) continue;
         const size_t r = (size_t)scan_to_raster(t0 + u, n, gh, gw, dir);
+        if (!index_ok(r < (size_t)n, err)) continue;
 #pragma unroll
         for (int w = 0; w < RJ; ++w) o[pv + r * DV + j0 + tj + 16 * w] = from_f32<T>(acc[a][w]);
     }
@@ -271,7 +268,7 @@ static int launch_generic_t(const Problem &p, void *ws, cudaStream_t st) {
     auto k1 = gla_chunk_state_kernel<T, DK, DV, C>;
     if (ensure_smem((const void *)k1, sm1)) return GTR_GLA_ERR_CUDA;
     k1<<<dim3(nc, bh), kGenThreads, sm1, st>>>((const T *)p.k, (const T *)p.v, p.la, dS, gam,
-                                               p.n, p.gh, p.gw, p.dir, nc);
+                                               p.n, p.gh, p.gw, p.dir, nc, p.err);
     note_launch();
 
     auto k2 = gla_state_scan_kernel<DK, DV>;
@@ -286,7 +283,7 @@ static int launch_generic_t(const Problem &p, void *ws, cudaStream_t st) {
     if (ensure_smem((const void *)k3, sm3)) return GTR_GLA_ERR_CUDA;
     k3<<<dim3(nc, bh, DV / VT), kGenThreads, sm3, st>>>((const T *)p.q, (const T *)p.k,
                                                          (const T *)p.v, p.la, dS, (T *)p.out,
-                                                         p.n, p.gh, p.gw, p.dir, nc);
+                                                         p.n, p.gh, p.gw, p.dir, nc, p.err);
     note_launch();
     return cudaPeekAtLastError() == cudaSuccess ? GTR_GLA_OK : GTR_GLA_ERR_CUDA;
 }

@@ -19,6 +19,13 @@ struct Problem {
     float *final_state;  // may be null
     int B, H, gh, gw, n, dk, dv, dir, dtype, chunk;
     int *err;            // device error word of the current device
+    // output tail fused into the stores (gtr_gla_fwd_tail): y = RMSNorm(o) w_n
+    // * SiLU(z), heads merged [B, N, H d_v]; `out` is then not written
+    int tail = 0;
+    const void *z = nullptr;
+    const float *wn = nullptr;
+    void *y = nullptr;
+    float eps = 0.f;
 };
 
 // Every workspace starts with a fixed header that only the fused kernel uses
@@ -57,5 +64,12 @@ int error_word(int **out);
 // Three-phase CUDA-core path (gla_generic.cu): all dtypes, chunk 32 or 64.
 size_t generic_workspace_bytes(const Problem &p);
 int launch_generic(const Problem &p, void *ws, cudaStream_t st);
+
+// Spatial SwiGLU block after its argument checks (swiglu.cu), with an optional
+// residual: y = resid + SwiGLU(x) (resid and y may be the same tensor).  The
+// workspace holds at least gtr_swiglu_workspace_size bytes.
+int swiglu_apply(const void *x, const void *w_gu, const float *b_gu, const float *w_dw, const float *b_dw,
+                 const void *w_down, const float *b_down, const void *resid, void *y, int B, int grid_h,
+                 int grid_w, int C, int F, int dtype, void *workspace, cudaStream_t stream);
 
 }  // namespace gtr

@@ -5,6 +5,7 @@
 #include <map>
 #include <mutex>
 
+#include "../../include/gtr_output_tail.h"
 #include "gla_common.cuh"
 #include "gla_internal.h"
 
@@ -201,6 +202,65 @@ int gtr_gla_fwd(const void *q, const void *k, const void *v, const float *log_al
     return dispatch(p, ws, stream);
 }
 
+// Output tail fused into the stores (d_k = d_v = 64), or for head sizes of 128
+// the attention into a workspace buffer followed by the tail kernel.
+static size_t tail_layout(const Problem &p, size_t *obuf) {
+    const size_t gla = workspace_bytes(p);
+    if (p.dk == 64 && p.dv == 64) {
+        *obuf = 0;
+        return gla;
+    }
+    *obuf = (gla + 255) & ~(size_t)255;
+    return *obuf + (size_t)p.B * p.H * p.n * p.dv * 2;
+}
+
+size_t gtr_gla_tail_workspace_size(int B, int H, int grid_h, int grid_w, int d_k, int d_v, int dtype) {
+    if (dtype != GTR_GLA_F16 && dtype != GTR_GLA_BF16) return 0;
+    if (validate_shape(B, H, grid_h, grid_w, d_k, d_v, dtype, 64)) return 0;
+    Problem p = make_problem(nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, B, H, grid_h, grid_w,
+                             d_k, d_v, 0, dtype, 64);
+    size_t obuf;
+    return tail_layout(p, &obuf);
+}
+
+int gtr_gla_fwd_tail(const void *q, const void *k, const void *v, const float *log_alpha, const void *z,
+                     const float *w_n, float eps, void *y, float *final_state, int B, int H, int grid_h,
+                     int grid_w, int d_k, int d_v, int direction, int dtype, void *workspace,
+                     size_t workspace_bytes_, cudaStream_t stream) {
+    if (dtype != GTR_GLA_F16 && dtype != GTR_GLA_BF16) return GTR_GLA_ERR_DTYPE;
+    // y takes the place of `out` in the checks: the same bytes, the same aliasing rules
+    Problem p = make_problem(q, k, v, log_alpha, y, final_state, B, H, grid_h, grid_w, d_k, d_v,
+                             direction, dtype, 64);
+    if (!z || !w_n) return GTR_GLA_ERR_NULL;
+    int rc = validate(p);
+    if (rc) return rc;
+    if (!(eps >= 0.f) || eps > 3.0e38f) return GTR_GLA_ERR_SHAPE;
+    if (misaligned(z) || misaligned(w_n)) return GTR_GLA_ERR_ALIGN;
+    const size_t ny = (size_t)p.B * p.H * p.n * p.dv * 2;
+    if (overlaps(y, ny, z, ny) || overlaps(y, ny, w_n, (size_t)p.H * p.dv * 4) ||
+        (final_state && overlaps(final_state, (size_t)p.B * p.H * p.dk * p.dv * 4, z, ny)))
+        return GTR_GLA_ERR_ALIAS;
+    size_t obuf;
+    const size_t need = tail_layout(p, &obuf);
+    if (!workspace || workspace_bytes_ < need || ((uintptr_t)workspace & 255u)) return GTR_GLA_ERR_WORKSPACE;
+    if (overlaps(y, ny, workspace, need)) return GTR_GLA_ERR_ALIAS;
+    int dev;
+    if ((rc = current_device(&dev))) return rc;
+    if ((rc = device_err_ptr(dev, &p.err))) return rc;
+    if (p.dk == 64 && p.dv == 64) {
+        p.tail = 1;
+        p.z = z;
+        p.wn = w_n;
+        p.y = y;
+        p.eps = eps;
+        return launch_fused(p, workspace, stream);
+    }
+    void *o = static_cast<char *>(workspace) + obuf;
+    p.out = o;
+    if ((rc = dispatch(p, workspace, stream))) return rc;
+    return gtr_output_tail_fwd(o, z, w_n, y, B, H, grid_h, grid_w, d_v, eps, dtype, stream);
+}
+
 size_t gtr_gla_workspace_size(int B, int H, int grid_h, int grid_w, int d_k, int d_v,
                               int dtype, int chunk) {
     if (validate_shape(B, H, grid_h, grid_w, d_k, d_v, dtype, chunk)) return 0;
@@ -223,7 +283,7 @@ int gtr_gla_status(cudaStream_t stream) {
         return GTR_GLA_ERR_CUDA;
     if (host_err == kDevErrTimeout) return GTR_GLA_ERR_TIMEOUT;
     if (host_err == kDevErrWorkspace) return GTR_GLA_ERR_WORKSPACE_STATE;
-    if (host_err == kDevErrRange) return GTR_GLA_ERR_RANGE;
+    if (host_err == kDevErrBounds) return GTR_GLA_ERR_BOUNDS;
     return host_err ? GTR_GLA_ERR_CUDA : GTR_GLA_OK;
 }
 
@@ -243,8 +303,7 @@ const char *gtr_gla_strerror(int code) {
         case GTR_GLA_ERR_ALIAS: return "output overlaps an input";
         case GTR_GLA_ERR_WORKSPACE_STATE:
             return "workspace header not zero when a call started (overlapping calls sharing it?)";
-        case GTR_GLA_ERR_RANGE:
-            return "a carried state exceeded the fp16 operand range (the output is not exact)";
+        case GTR_GLA_ERR_BOUNDS: return "a kernel's index check failed (checked build)";
         default: return "unknown error code";
     }
 }

@@ -19,19 +19,6 @@
 namespace gtr {
 namespace {
 
-__device__ __forceinline__ float tanh_hw(float x) {
-    float y;
-    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
-// SiLU(z) = z * sigmoid(z) = z/2 * (1 + tanh(z/2)): one hardware tanh (relative
-// error about 2^-11, that of the fp16 rounding of the result).
-__device__ __forceinline__ float silu(float z) {
-    const float hz = 0.5f * z;
-    return fmaf(hz, tanh_hw(hz), hz);
-}
-
 // One thread per 8 channels of a token-head; L = d_v / 8 consecutive lanes
 // share a token-head, token-heads ordered (image, token, head) with the head
 // fastest, so a warp's z and y accesses are contiguous.  Grid-stride over
@@ -73,8 +60,8 @@ __global__ void __launch_bounds__(256, 8)
             uint32_t out[4];
 #pragma unroll
             for (int q = 0; q < 4; ++q)
-                out[q] = Pair<T>::pack(of[q].x * r * wv[2 * q] * silu(zf[q].x),
-                                       of[q].y * r * wv[2 * q + 1] * silu(zf[q].y));
+                out[q] = Pair<T>::pack(of[q].x * r * wv[2 * q] * silu_f32(zf[q].x),
+                                       of[q].y * r * wv[2 * q + 1] * silu_f32(zf[q].y));
             *reinterpret_cast<uint4 *>(y + th * DV + 8 * l) = make_uint4(out[0], out[1], out[2], out[3]);
         }
     }

@@ -56,20 +56,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
-// try_wait with a suspend-time hint: a thread whose phase is not complete
-// sleeps in hardware until it completes or about `hint_ns` have passed.
-__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
-        : "memory");
-    return ok != 0;
-}
-
 // Non-blocking probe of an mbarrier phase.
 __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
@@ -127,14 +113,6 @@ __device__ __forceinline__ void tma_load_4d_pol(void *dst, const CUtensorMap *ma
         "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar)),
         "l"(pol)
         : "memory");
-}
-
-// Bring the box of a 3-D tile at (c0, c1, c2) into L2 (no shared-memory destination).
-__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap *map, int c0, int c1, int c2) {
-    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
-                     reinterpret_cast<uint64_t>(map)),
-                 "r"(c0), "r"(c1), "r"(c2)
-                 : "memory");
 }
 
 // Row gather with an L2 cache policy: four rows (r0..r3) of a 2-D tensor whose
@@ -293,22 +271,6 @@ __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
         : "=l"(d)
         : "l"(*reinterpret_cast<const uint64_t *>(&a)), "l"(*reinterpret_cast<const uint64_t *>(&b)),
           "l"(*reinterpret_cast<const uint64_t *>(&c)));
-    return *reinterpret_cast<float2 *>(&d);
-}
-
-__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
-    uint64_t d;
-    asm("add.rn.f32x2 %0, %1, %2;"
-        : "=l"(d)
-        : "l"(*reinterpret_cast<const uint64_t *>(&a)), "l"(*reinterpret_cast<const uint64_t *>(&b)));
-    return *reinterpret_cast<float2 *>(&d);
-}
-
-__device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
-    uint64_t d;
-    asm("sub.rn.f32x2 %0, %1, %2;"
-        : "=l"(d)
-        : "l"(*reinterpret_cast<const uint64_t *>(&a)), "l"(*reinterpret_cast<const uint64_t *>(&b)));
     return *reinterpret_cast<float2 *>(&d);
 }
 

@@ -7,8 +7,6 @@
 // "GTR: Gated Token Recurrence for Efficient Dense Prediction", x-techcon
 // article, section 架构: a SwiGLU whose value branch gets a 3 x 3 per-channel
 // convolution, so that neighbouring patches exchange information directly.
-#include <cublasLt.h>
-
 #include <map>
 #include <mutex>
 #include <tuple>
@@ -17,6 +15,7 @@
 #include "gla_common.cuh"
 #include "gla_internal.h"
 #include "io_pack.cuh"
+#include "lt_gemm.h"
 #include "sm100.cuh"
 
 namespace gtr {
@@ -291,84 +290,6 @@ __global__ void add_bias_kernel(T *y, const float *bias, size_t M, int C) {
     *p = Pair<T>::pack(o.x + bias[c], o.y + bias[c + 1]);
 }
 
-// ---------------------------------------------------------------- cuBLASLt
-
-constexpr size_t kLtWorkspace = 32u << 20;
-
-struct LtPlan {
-    cublasLtMatmulDesc_t op = nullptr;
-    cublasLtMatrixLayout_t a = nullptr, b = nullptr, d = nullptr;
-    cublasLtMatmulAlgo_t algo;
-    bool ok = false;
-};
-
-std::mutex g_lt_mu;
-cublasLtHandle_t g_lt[64];
-std::map<std::tuple<int, int, long long, int, int, bool>, LtPlan> g_plans;
-
-// out[M, N] (row-major) = in[M, K] (row-major) . W[N, K]^T (+ bias[N], output type).
-// In cuBLASLt's column-major terms: out^T (N x M) = W (N x K) . in^T (K x M),
-// with W stored as a K x N column-major matrix (transposed in the op).
-// Called with g_lt_mu held.
-int lt_plan(int dev, int dtype, long long M, int N, int K, bool bias, LtPlan **out) {
-    if (!g_lt[dev] && cublasLtCreate(&g_lt[dev]) != CUBLAS_STATUS_SUCCESS) return GTR_GLA_ERR_CUDA;
-    auto key = std::make_tuple(dev, dtype, M, N, K, bias);
-    auto it = g_plans.find(key);
-    if (it != g_plans.end()) {
-        *out = &it->second;
-        return it->second.ok ? GTR_GLA_OK : GTR_GLA_ERR_CUDA;
-    }
-    LtPlan &pl = g_plans[key];
-    const cudaDataType_t dt = dtype == GTR_GLA_BF16 ? CUDA_R_16BF : CUDA_R_16F;
-    bool good = cublasLtMatmulDescCreate(&pl.op, CUBLAS_COMPUTE_32F, CUDA_R_32F) == CUBLAS_STATUS_SUCCESS;
-    const cublasOperation_t opT = CUBLAS_OP_T, opN = CUBLAS_OP_N;
-    good = good && cublasLtMatmulDescSetAttribute(pl.op, CUBLASLT_MATMUL_DESC_TRANSA, &opT, sizeof(opT)) ==
-                       CUBLAS_STATUS_SUCCESS;
-    good = good && cublasLtMatmulDescSetAttribute(pl.op, CUBLASLT_MATMUL_DESC_TRANSB, &opN, sizeof(opN)) ==
-                       CUBLAS_STATUS_SUCCESS;
-    if (bias) {  // bias vector in the output type
-        const cublasLtEpilogue_t epi = CUBLASLT_EPILOGUE_BIAS;
-        good = good && cublasLtMatmulDescSetAttribute(pl.op, CUBLASLT_MATMUL_DESC_EPILOGUE, &epi, sizeof(epi)) ==
-                           CUBLAS_STATUS_SUCCESS;
-    }
-    good = good && cublasLtMatrixLayoutCreate(&pl.a, dt, K, N, K) == CUBLAS_STATUS_SUCCESS;
-    good = good && cublasLtMatrixLayoutCreate(&pl.b, dt, K, M, K) == CUBLAS_STATUS_SUCCESS;
-    good = good && cublasLtMatrixLayoutCreate(&pl.d, dt, N, M, N) == CUBLAS_STATUS_SUCCESS;
-    cublasLtMatmulPreference_t pref = nullptr;
-    good = good && cublasLtMatmulPreferenceCreate(&pref) == CUBLAS_STATUS_SUCCESS;
-    const size_t wsb = kLtWorkspace;
-    good = good && cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MAX_WORKSPACE_BYTES, &wsb,
-                                                        sizeof(wsb)) == CUBLAS_STATUS_SUCCESS;
-    cublasLtMatmulHeuristicResult_t res;
-    int n = 0;
-    good = good && cublasLtMatmulAlgoGetHeuristic(g_lt[dev], pl.op, pl.a, pl.b, pl.d, pl.d, pref, 1, &res, &n) ==
-                       CUBLAS_STATUS_SUCCESS &&
-           n > 0;
-    if (pref) cublasLtMatmulPreferenceDestroy(pref);
-    if (good) pl.algo = res.algo;
-    pl.ok = good;
-    *out = &pl;
-    return good ? GTR_GLA_OK : GTR_GLA_ERR_CUDA;
-}
-
-int lt_gemm(int dev, int dtype, long long M, int N, int K, const void *in, const void *w, const void *bias,
-            void *out, void *lt_ws, cudaStream_t st) {
-    // one lock across the plan lookup, the bias pointer (an attribute of the
-    // shared descriptor) and the enqueue
-    std::lock_guard<std::mutex> lock(g_lt_mu);
-    LtPlan *pl;
-    int rc = lt_plan(dev, dtype, M, N, K, bias != nullptr, &pl);
-    if (rc) return rc;
-    if (bias && cublasLtMatmulDescSetAttribute(pl->op, CUBLASLT_MATMUL_DESC_BIAS_POINTER, &bias,
-                                               sizeof(bias)) != CUBLAS_STATUS_SUCCESS)
-        return GTR_GLA_ERR_CUDA;
-    const float one = 1.f, zero = 0.f;
-    return cublasLtMatmul(g_lt[dev], pl->op, &one, w, pl->a, in, pl->b, &zero, out, pl->d, out, pl->d,
-                          &pl->algo, lt_ws, kLtWorkspace, st) == CUBLAS_STATUS_SUCCESS
-               ? GTR_GLA_OK
-               : GTR_GLA_ERR_CUDA;
-}
-
 struct SwLayout {
     size_t gu, h, bd, lt, total;
 };
@@ -457,6 +378,46 @@ int launch_dw_gate(int dtype, const void *gu, const float *b_gu, const float *w_
 }
 
 }  // namespace
+
+// The block after argument checks (shared with the backbone layer): y = x +
+// ... when resid = x is given (the down projection adds it as cuBLASLt's C
+// operand; y may be x itself).
+int swiglu_apply(const void *x, const void *w_gu, const float *b_gu, const float *w_dw, const float *b_dw,
+                 const void *w_down, const float *b_down, const void *resid, void *y, int B, int grid_h,
+                 int grid_w, int C, int F, int dtype, void *workspace, cudaStream_t stream) {
+    const long long M = (long long)B * grid_h * grid_w;
+    const SwLayout l = sw_layout(M, C, F, 2);
+    int rc;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return GTR_GLA_ERR_CUDA;
+    char *ws = static_cast<char *>(workspace);
+    void *gu = ws + l.gu, *h = ws + l.h, *bd = ws + l.bd, *lt_ws = ws + l.lt;
+    // 1. [g | u] without biases (the kernel adds them in fp32)
+    rc = lt_gemm(dev, dtype, M, 2 * F, C, x, w_gu, nullptr, nullptr, gu, lt_ws, stream);
+    if (rc) return rc;
+    // 2. biases, depthwise 3 x 3 on the value branch, SiLU gate, product
+    rc = launch_dw_gate(dtype, gu, b_gu, w_dw, b_dw, h, b_down, bd, B, grid_h, grid_w, F, C, stream);
+    if (rc) return rc;
+    // 3. y = h W_d^T + b_d (the bias, copied to the I/O dtype by the kernel
+    //    above, in the GEMM's epilogue; one pass of this library in fp32 if
+    //    cuBLASLt offers no such epilogue)
+    rc = lt_gemm(dev, dtype, M, C, F, h, w_down, bd, resid, y, lt_ws, stream);
+    if (rc) {
+        rc = lt_gemm(dev, dtype, M, C, F, h, w_down, nullptr, resid, y, lt_ws, stream);
+        if (rc) return rc;
+        const size_t pairs = (size_t)M * C / 2;
+        const unsigned blocks = (unsigned)((pairs + 255) / 256);
+        if (dtype == GTR_GLA_BF16)
+            add_bias_kernel<__nv_bfloat16><<<blocks, 256, 0, stream>>>(static_cast<__nv_bfloat16 *>(y), b_down,
+                                                                       (size_t)M, C);
+        else
+            add_bias_kernel<__half><<<blocks, 256, 0, stream>>>(static_cast<__half *>(y), b_down, (size_t)M, C);
+        note_launch();
+        if (cudaPeekAtLastError() != cudaSuccess) return GTR_GLA_ERR_CUDA;
+    }
+    return GTR_GLA_OK;
+}
+
 }  // namespace gtr
 
 using namespace gtr;
@@ -487,32 +448,6 @@ extern "C" int gtr_swiglu_fwd(const void *x, const void *w_gu, const float *b_gu
     const SwLayout l = sw_layout(M, C, F, es);
     if (!workspace || workspace_bytes < l.total || ((uintptr_t)workspace & 255u)) return GTR_GLA_ERR_WORKSPACE;
     if (overlap(y, ny, workspace, l.total)) return GTR_GLA_ERR_ALIAS;
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return GTR_GLA_ERR_CUDA;
-    char *ws = static_cast<char *>(workspace);
-    void *gu = ws + l.gu, *h = ws + l.h, *bd = ws + l.bd, *lt_ws = ws + l.lt;
-    // 1. [g | u] without biases (the kernel adds them in fp32)
-    rc = lt_gemm(dev, dtype, M, 2 * F, C, x, w_gu, nullptr, gu, lt_ws, stream);
-    if (rc) return rc;
-    // 2. biases, depthwise 3 x 3 on the value branch, SiLU gate, product
-    rc = launch_dw_gate(dtype, gu, b_gu, w_dw, b_dw, h, b_down, bd, B, grid_h, grid_w, F, C, stream);
-    if (rc) return rc;
-    // 3. y = h W_d^T + b_d (the bias, copied to the I/O dtype by the kernel
-    //    above, in the GEMM's epilogue; one pass of this library in fp32 if
-    //    cuBLASLt offers no such epilogue)
-    rc = lt_gemm(dev, dtype, M, C, F, h, w_down, bd, y, lt_ws, stream);
-    if (rc) {
-        rc = lt_gemm(dev, dtype, M, C, F, h, w_down, nullptr, y, lt_ws, stream);
-        if (rc) return rc;
-        const size_t pairs = (size_t)M * C / 2;
-        const unsigned blocks = (unsigned)((pairs + 255) / 256);
-        if (dtype == GTR_GLA_BF16)
-            add_bias_kernel<__nv_bfloat16><<<blocks, 256, 0, stream>>>(static_cast<__nv_bfloat16 *>(y), b_down,
-                                                                       (size_t)M, C);
-        else
-            add_bias_kernel<__half><<<blocks, 256, 0, stream>>>(static_cast<__half *>(y), b_down, (size_t)M, C);
-        note_launch();
-        if (cudaPeekAtLastError() != cudaSuccess) return GTR_GLA_ERR_CUDA;
-    }
-    return GTR_GLA_OK;
+    return swiglu_apply(x, w_gu, b_gu, w_dw, b_dw, w_down, b_down, nullptr, y, B, grid_h, grid_w, C, F, dtype,
+                        workspace, stream);
 }

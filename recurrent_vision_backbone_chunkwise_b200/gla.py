@@ -33,6 +33,10 @@ _lib.gtr_gla_fwd_ex.argtypes = [_vp] * 6 + [_int] * 9 + [_vp, _sz, _vp]
 _lib.gtr_gla_fwd_ex.restype = _int
 _lib.gtr_gla_fwd_noalloc.argtypes = [_vp] * 6 + [_int] * 7 + [_vp]
 _lib.gtr_gla_fwd_noalloc.restype = _int
+_lib.gtr_gla_fwd_tail.argtypes = [_vp] * 6 + [ctypes.c_float] + [_vp] * 2 + [_int] * 8 + [_vp, _sz, _vp]
+_lib.gtr_gla_fwd_tail.restype = _int
+_lib.gtr_gla_tail_workspace_size.argtypes = [_int] * 7
+_lib.gtr_gla_tail_workspace_size.restype = _sz
 _lib.gtr_gla_workspace_size.argtypes = [_int] * 8
 _lib.gtr_gla_workspace_size.restype = _sz
 _lib.gtr_gla_status.argtypes = [_vp]
@@ -188,3 +192,38 @@ def gtr_gla_fwd_noalloc(q, k, v, log_alpha, direction, out, final_state=None, st
     if rc != 0:
         raise GlaError(rc)
     return out, final_state
+
+
+def gtr_gla_tail_workspace_size(B, H, grid_h, grid_w, d_k, d_v, dtype=F16) -> int:
+    return int(_lib.gtr_gla_tail_workspace_size(B, H, grid_h, grid_w, d_k, d_v, dtype))
+
+
+def gtr_gla_fwd_tail(q, k, v, log_alpha, z, w_n, direction, eps=1e-5, y=None, final_state=None,
+                     want_state=True, workspace=None, stream=None):
+    """Forward pass with the output tail fused into its stores: y [B, grid_h,
+    grid_w, H*d_v] = RMSNorm_head(o) * w_n * SiLU(z), fp16 or bf16 (dtype of q).
+    A workspace is allocated (zero-filled) if not given.  Returns (y, final_state)."""
+    _validate(q, k, v, log_alpha, None, final_state)
+    B, H, gh, gw, dk, dv = _shape(q, v)
+    if q.dtype not in (torch.float16, torch.bfloat16):
+        raise ValueError("gtr_gla_fwd_tail takes fp16 or bf16 q, k, v")
+    dev = q.device
+    _check("z", z, (B, gh, gw, H * dv), q.dtype, dev)
+    _check("w_n", w_n, (H, dv), torch.float32, dev)
+    if y is None:
+        y = torch.empty((B, gh, gw, H * dv), dtype=q.dtype, device=dev)
+    _check("y", y, (B, gh, gw, H * dv), q.dtype, dev)
+    if final_state is None and want_state:
+        final_state = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    dtype = _DTYPE_CODE[q.dtype]
+    need = gtr_gla_tail_workspace_size(B, H, gh, gw, dk, dv, dtype)
+    if workspace is None:
+        workspace = torch.zeros(max(need, 1), dtype=torch.uint8, device=dev)
+    _check("workspace", workspace, (workspace.numel(),), torch.uint8, dev)
+    rc = _lib.gtr_gla_fwd_tail(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(z), _ptr(w_n),
+                               float(eps), _ptr(y), _ptr(final_state), B, H, gh, gw, dk, dv,
+                               int(direction), dtype, _ptr(workspace), workspace.numel(),
+                               _vp(_stream_handle(stream)))
+    if rc != 0:
+        raise GlaError(rc)
+    return y, final_state

@@ -26,7 +26,7 @@ def declared_functions():
     for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
         text = open(h).read()
         text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-        for m in re.finditer(r"\b(gtr_(?:gla|swiglu|output_tail)_\w+)\s*\(", text):
+        for m in re.finditer(r"\b(gtr_(?:gla|swiglu|output_tail|layer|backbone)_\w+)\s*\(", text):
             names.add(m.group(1))
     return sorted(names)
 
@@ -35,7 +35,8 @@ def test_header_declares_entry_points():
     names = declared_functions()
     for n in ("gtr_gla_fwd", "gtr_gla_fwd_ex", "gtr_gla_workspace_size", "gtr_gla_status",
               "gtr_gla_strerror", "gtr_gla_release", "gtr_gla_launch_count",
-              "gtr_swiglu_fwd", "gtr_swiglu_workspace_size", "gtr_output_tail_fwd"):
+              "gtr_swiglu_fwd", "gtr_swiglu_workspace_size", "gtr_output_tail_fwd",
+              "gtr_layer_fwd", "gtr_backbone_fwd", "gtr_layer_workspace_size"):
         assert n in names
 
 
@@ -44,9 +45,10 @@ def test_library_exports_every_declared_symbol(gla):
     for n in declared_functions():
         assert hasattr(lib, n), f"{n} declared in include/ but not exported"
         # the binding forwards under the same name
-        from recurrent_vision_backbone_chunkwise_b200 import output_tail, swiglu
+        from recurrent_vision_backbone_chunkwise_b200 import layer, output_tail, swiglu
 
-        mod = swiglu if n.startswith("gtr_swiglu_") else output_tail if n.startswith("gtr_output_tail_") else gla
+        mod = (swiglu if n.startswith("gtr_swiglu_") else output_tail if n.startswith("gtr_output_tail_")
+               else layer if n.startswith(("gtr_layer_", "gtr_backbone_")) else gla)
         assert hasattr(mod, n), n
 
 
@@ -54,7 +56,7 @@ def test_strerror_and_count(gla):
     assert gla.gtr_gla_strerror(0) == "ok"
     assert "direction" in gla.gtr_gla_strerror(-4)
     assert gla.gtr_gla_strerror(12345) == "unknown error code"
-    for code in range(-12, 0):  # every declared code has its own text
+    for code in range(-13, 0):  # every declared code has its own text
         assert gla.gtr_gla_strerror(code) != "unknown error code", code
     assert "workspace header" in gla.gtr_gla_strerror(-12)
     assert "timed out" in gla.gtr_gla_strerror(-10)
@@ -66,9 +68,10 @@ def test_workspace_size(gla):
     # invalid shapes report 0
     assert gla.gtr_gla_workspace_size(0, 6, 40, 40, 64, 64, gla.F16, 64) == 0
     assert gla.gtr_gla_workspace_size(1, 6, 40, 40, 48, 64, gla.F16, 64) == 0
-    a = gla.gtr_gla_workspace_size(1, 12, 128, 128, 64, 64, gla.F16, 64)
-    b = gla.gtr_gla_workspace_size(2, 12, 128, 128, 64, 64, gla.F16, 64)
-    assert b >= a
+    # the header (64 KiB) at least; beyond it the size follows the segment plan
+    # (which may hold fewer segment states for more planes), not the batch
+    for B in (1, 2, 8):
+        assert gla.gtr_gla_workspace_size(B, 12, 128, 128, 64, 64, gla.F16, 64) >= 65536
 
 
 # fake, 256-aligned, non-overlapping "device" addresses; never dereferenced
@@ -208,3 +211,103 @@ def test_binding_checks_tensors_before_any_call(gla, bad):
     with pytest.raises(ValueError):
         gla.gtr_gla_fwd_noalloc(q, k, v, la, 0, out if out is not None else torch.zeros_like(v), fs)
     assert gla.gtr_gla_launch_count() == before
+
+
+# ---------------------------------------------------------------- backbone layer
+
+def _layer_struct(layer, base=0x40000000, **override):
+    vals = {n: base + 0x100000 * i for i, n in enumerate(layer._FIELDS)}
+    vals.update(override)
+    return layer.GtrLayerWeights(*[ctypes.c_void_p(vals[n]) for n in layer._FIELDS])
+
+
+def call_layer(gla, **kw):
+    from recurrent_vision_backbone_chunkwise_b200 import layer
+
+    a = dict(x=0x20000000, w=_layer_struct(layer), B=1, gh=6, gw=7, C=128, F=512, dir=0,
+             dtype=gla.F16, ws=0x30000000, wsb=1 << 34)
+    a.update(kw)
+    w = a["w"]
+    return gla._lib.gtr_layer_fwd(ctypes.c_void_p(a["x"]), None if w is None else ctypes.byref(w), a["B"],
+                                  a["gh"], a["gw"], a["C"], a["F"], a["dir"], a["dtype"],
+                                  ctypes.c_void_p(a["ws"]), a["wsb"], None)
+
+
+def test_layer_workspace_size(gla):
+    from recurrent_vision_backbone_chunkwise_b200 import layer
+
+    a = layer.gtr_layer_workspace_size(1, 40, 40, 384, 1536, gla.F16)
+    assert a > 0 and layer.gtr_layer_workspace_size(8, 40, 40, 384, 1536, gla.F16) > a
+    assert layer.gtr_layer_workspace_size(1, 40, 40, 100, 400, gla.F16) == 0  # C not a multiple of 64
+    assert layer.gtr_layer_workspace_size(1, 40, 40, 128, 0, gla.F16) == 0
+    assert layer.gtr_layer_workspace_size(1, 40, 40, 128, 512, gla.F32) == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(x=0), -1), (dict(w=None), -1), ("w_o_null", -1),
+    (dict(C=100), -2), (dict(C=4096), -2), (dict(F=0), -2), (dict(F=12), -2), (dict(B=0), -2),
+    (dict(dir=4), -4), (dict(dtype=2), -6), (dict(x=0x20000008), -5), ("w_gu_misaligned", -5),
+    (dict(ws=0), -8), (dict(wsb=1024), -8), (dict(ws=0x30000010), -8),
+])
+def test_layer_argument_errors(gla, kw, code):
+    from recurrent_vision_backbone_chunkwise_b200 import layer
+
+    if kw == "w_o_null":
+        kw = dict(w=_layer_struct(layer, w_o=0))
+    elif kw == "w_gu_misaligned":
+        kw = dict(w=_layer_struct(layer, w_gu=0x50000004))
+    assert call_layer(gla, **kw) == code
+
+
+def test_backbone_argument_errors(gla):
+    from recurrent_vision_backbone_chunkwise_b200 import layer
+
+    arr = (layer.GtrLayerWeights * 2)(_layer_struct(layer), _layer_struct(layer, b_dw=0))
+    vp = ctypes.c_void_p
+    f = gla._lib.gtr_backbone_fwd
+    assert f(vp(0x20000000), arr, 2, 1, 6, 7, 128, 512, gla.F16, vp(0x30000000), 1 << 34, None) == -1
+    assert f(vp(0x20000000), None, 2, 1, 6, 7, 128, 512, gla.F16, vp(0x30000000), 1 << 34, None) == -1
+    assert f(vp(0x20000000), arr, 0, 1, 6, 7, 128, 512, gla.F16, vp(0x30000000), 1 << 34, None) == -2
+    assert f(vp(0x20000000), arr, 1, 1, 6, 7, 128, 512, gla.F16, vp(0x30000000), 1024, None) == -8
+
+
+# ------------------------------------------------------------ fused output tail
+
+def call_tail(gla, **kw):
+    a = dict(q=Q, k=K, v=V, la=LA, z=0x80000000, w=0x90000000, eps=1e-5, y=OUT, fs=FS, B=1, H=2, gh=4,
+             gw=4, dk=64, dv=64, dir=0, dtype=gla.F16, ws=WS, wsb=1 << 30)
+    a.update(kw)
+    vp = ctypes.c_void_p
+    return gla._lib.gtr_gla_fwd_tail(vp(a["q"]), vp(a["k"]), vp(a["v"]), vp(a["la"]), vp(a["z"]), vp(a["w"]),
+                                     a["eps"], vp(a["y"]), vp(a["fs"]), a["B"], a["H"], a["gh"], a["gw"],
+                                     a["dk"], a["dv"], a["dir"], a["dtype"], vp(a["ws"]), a["wsb"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(z=0), -1), (dict(w=0), -1), (dict(y=0), -1), (dict(q=0), -1),
+    (dict(eps=-1.0), -2), (dict(eps=float("nan")), -2), (dict(eps=float("inf")), -2), (dict(B=0), -2),
+    (dict(dk=48), -3), (dict(dir=5), -4), (dict(z=0x80000008), -5), (dict(w=0x90000004), -5),
+    (dict(dtype=2), -6), (dict(wsb=0), -8), (dict(ws=0), -8),
+    (dict(z=OUT + 64), -11), (dict(y=Q), -11), (dict(w=OUT + 256), -11),
+])
+def test_tail_argument_errors(gla, kw, code):
+    assert call_tail(gla, **kw) == code
+
+
+def test_tail_workspace_size(gla):
+    a = gla.gtr_gla_tail_workspace_size(1, 6, 40, 40, 64, 64, gla.F16)
+    assert a == gla.gtr_gla_workspace_size(1, 6, 40, 40, 64, 64, gla.F16, 64)  # fused: no o buffer
+    b = gla.gtr_gla_tail_workspace_size(1, 6, 40, 40, 128, 128, gla.F16)
+    assert b >= gla.gtr_gla_workspace_size(1, 6, 40, 40, 128, 128, gla.F16, 64) + 1600 * 6 * 128 * 2
+    assert gla.gtr_gla_tail_workspace_size(1, 6, 40, 40, 64, 64, gla.F32) == 0
+
+
+def test_checked_build_exports_every_declared_symbol(gla):
+    from recurrent_vision_backbone_chunkwise_b200 import build
+
+    path = build.build(checked=True)
+    lib = ctypes.CDLL(path)
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+    lib.gtr_gla_strerror.restype = ctypes.c_char_p
+    assert b"index check" in lib.gtr_gla_strerror(-13)
