@@ -244,7 +244,7 @@ def run_swiglu(args):
                      "frac": achieved / peak, "traffic": None,
                      "peak_source": f"{peak_kind} dense bf16 burst",
                      "flops_per_call": flops,
-                     "timed_unit": "one block: two cuBLASLt projections and the fused kernel"},
+                     "timed_unit": "one block: the two tensor-core GEMMs and the fused kernel"},
         "gpu_launches": int(launches),
         "e2e": {"value": aggregate_rate(ri.world, K2, M, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": M * C * 2, "d2h_bytes_per_step": M * C * 2, "steps": K2},

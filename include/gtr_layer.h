@@ -33,15 +33,15 @@
  * activations, the GLA's scratch and the GEMM scratch; calls sharing one must
  * be stream-ordered.
  * Calls are asynchronous and stream-ordered; device-side GLA errors are read
- * by gtr_gla_status.  The projections run on cuBLASLt; everything else in
- * kernels of this library.
+ * by gtr_gla_status.  Every step runs in this library's kernels (the
+ * projections on its tensor-core GEMM, gtr_gemm.h).
  *
  * Errors (codes of gtr_gla.h, reported before anything is launched):
  * GTR_GLA_ERR_NULL (x, w or any weight pointer NULL), _SHAPE (B, grid <= 0,
  * C not a positive multiple of 64 or above 2048, F <= 0 or not a multiple of
  * 8, too many tokens, n_layers < 1), _DIRECTION, _DTYPE, _ALIGN (a pointer not
  * 16-byte aligned), _WORKSPACE (NULL, too small or not 256-byte aligned),
- * _CUDA (a launch or cuBLASLt call failed).
+ * _CUDA (a launch failed).
  */
 #ifndef GTR_LAYER_H
 #define GTR_LAYER_H

@@ -25,15 +25,15 @@
  *   b_down  [C]                      fp32
  *   y       [B, grid_h, grid_w, C]   I/O dtype, must not overlap any input
  * C and F must be multiples of 8 and every pointer 16-byte aligned.  The two
- * projections are dense GEMMs run by cuBLASLt on the tensor cores (fp32
- * accumulation); b_g, b_u, b_dw, the depthwise convolution, the SiLU gate and
+ * projections run on this library's tensor-core GEMM (gtr_gemm.h: tcgen05,
+ * fp32 accumulation); b_g, b_u, b_dw, the depthwise convolution, the SiLU gate and
  * the product run in this library's own kernel, in fp32, between them; b_down
  * is rounded once to the I/O dtype and added in fp32 in the down projection's
  * epilogue.  The projected gate/value and the gated product are kept in the
  * workspace in the I/O dtype.
  *
- * Return codes are those of gtr_gla.h; GTR_GLA_ERR_CUDA also covers a
- * cuBLASLt failure.  Calls are asynchronous and stream-ordered.
+ * Return codes are those of gtr_gla.h.  Calls are asynchronous and
+ * stream-ordered.
  */
 #ifndef GTR_SWIGLU_H
 #define GTR_SWIGLU_H

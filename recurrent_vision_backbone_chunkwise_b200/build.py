@@ -31,8 +31,7 @@ BUILD_CHECKED = os.path.join(PKG, "_build_checked")
 LIB_CHECKED = os.path.join(PKG, "libgtr_gla_checked.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
-# cuBLASLt runs the dense projections of the Spatial SwiGLU block
-LINK = ["-lcublasLt", "-Xlinker", "-rpath=/usr/local/cuda/lib64"]
+LINK = ["-Xlinker", "-rpath=/usr/local/cuda/lib64"]
 NVFLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
            "--expt-relaxed-constexpr", "-I", os.path.join(ROOT, "include")]
 

@@ -97,10 +97,20 @@ constexpr uint32_t MISC_FLAG = 1552;  // int   [kStages] exact-score chunk
 constexpr uint32_t MISC_TOT = 2048;   // float [2][kOpWarps][64] operand warps' row-block log sums
 constexpr uint32_t MISC_TAIL = 6144;  // float [2][2][64] output tail: half-row sums of squares
 constexpr uint32_t MISC_BYTES = 8192;
-constexpr uint32_t SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
+// gate totals of the plane's segments, staged for the transposed scan
+constexpr uint32_t OFF_SCAN = OFF_MISC + MISC_BYTES;
+constexpr uint32_t SCAN_BYTES = 8192;
+constexpr int kMaxScanSegments = 33;  // (P - 1) * 64 gate totals fit SCAN_BYTES
+constexpr uint32_t SMEM_BYTES = OFF_SCAN + SCAN_BYTES + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory");
 static_assert(MISC_TOT + 2 * kOpWarps * 64 * 4 <= MISC_TAIL && MISC_TAIL + 1024 <= MISC_BYTES, "misc area");
 static_assert(kMaxSegments * 64 * 4 <= 2 * 8192, "the fold stages every gate total in the A buffers");
+static_assert((kMaxScanSegments - 1) * 64 * 4 <= SCAN_BYTES, "scan gate totals");
+// the scan stages its slice of every aggregate, (2048 / P + 1) (P - 1) pairs,
+// in the A buffers
+static_assert((2048 / kMaxScanSegments + 1) * (kMaxScanSegments - 1) * 8 <= 2 * 8192, "scan slice");
+static_assert((kMaxScanSegments - 1) * 64 <= 8 * 256 && (2048 / kMaxScanSegments + 1) * (kMaxScanSegments - 1) <= 8 * 256,
+              "the scan's loads take one pass of the 256 epilogue threads");
 static_assert(FC % kOpWarps == 0 && FC / kOpWarps == 8, "operand warps own 8 tokens each");
 
 constexpr uint32_t kTmemCols = 512;
@@ -280,6 +290,9 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
+    unsigned arrival = 0;  // coop: this CTA's place in the arrival count (header check)
+    // (no descriptor prefetch: on B200 each prefetch.tensormap held the issuing
+    // thread for about 0.45 us; the first copy of each map fetches it anyway)
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&bar_full[s], 1);  // producer lane 0 (with the stage's TMA bytes)
@@ -298,7 +311,16 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
         mbar_init(&bar_fin, 1);
         mbar_init(&bar_pub, kEpiThreads);
         fence_mbar_init();
-        s_ticket = (int)atomicAdd(&p.ctr[0], 1u);
+        // A cooperative launch has every CTA resident, so the block index can
+        // name the segment; the arrival count is still kept (its value is
+        // only checked at the end, off the critical path).  Otherwise the
+        // ticket order guarantees that a CTA only waits for earlier ones.
+        if (p.coop) {
+            arrival = atomicAdd(&p.ctr[0], 1u);
+            s_ticket = (int)blockIdx.x;
+        } else {
+            s_ticket = (int)atomicAdd(&p.ctr[0], 1u);
+        }
         s_abort = 0;
     }
     for (int e = tid; e < kStages * 64; e += kThreads) sRows[e] = 0;
@@ -332,12 +354,6 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
         // FC / boxh column slabs per tensor for column scans.
         const uint64_t pol_keep = l2_policy_evict_last();  // pre-pass data is read again
         const uint64_t pol_once = l2_policy_evict_first();
-        if (lane == 0) {
-            tma_prefetch_desc(&p.tm_q);
-            tma_prefetch_desc(&p.tm_k);
-            tma_prefetch_desc(&p.tm_v);
-            tma_prefetch_desc(&p.tm_la);
-        }
         bool ok = true;
         uint32_t issued = 0;  // bit s: the last use of stage s had its copies issued
         for (int it = 0; it < n_items; ++it) {
@@ -773,29 +789,48 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
             }
             named_bar_sync(kBarEpi, kEpiThreads);
             if (s_abort) ok = false;
-            float *sGt = reinterpret_cast<float *>(sm + OFF_A);  // unused until the first mask
-            if (ok)
-                for (int e = et; e < (p.P - 1) * 64; e += kEpiThreads)
-                    sGt[e] = __ldcg(p.aggg + (size_t)bh * p.P * 64 + e);
-            named_bar_sync(kBarEpi, kEpiThreads);
+            // stage this CTA's slice of every aggregate (A buffers, unused until
+            // the first mask) and the plane's gate totals, every load in
+            // flight at once, then scan the slice's pairs through the segments
             const float2 *agp = reinterpret_cast<const float2 *>(p.agg + (size_t)bh * p.P * 4096);
             float2 *sinp = reinterpret_cast<float2 *>(p.sin + (size_t)bh * p.P * 4096);
+            float2 *sA = reinterpret_cast<float2 *>(sm + OFF_A);
+            float *sG = reinterpret_cast<float *>(sm + OFF_SCAN);
             const int u0 = seg * 2048 / p.P, u1 = (seg + 1) * 2048 / p.P;
-            if (ok && index_ok(bh < p.BH && seg < p.P && u1 <= 2048 && p.P <= kMaxSegments, p.err)) {
-                for (int u = u0 + et; u < u1; u += kEpiThreads) {
-                    const int i = (2 * u) & 63;  // key dim of the pair's first element
+            const int m = u1 - u0, nA = (p.P - 1) * m;
+            if (ok && !index_ok(bh < p.BH && seg < p.P && p.P <= kMaxScanSegments && u1 <= 2048, p.err)) ok = false;
+            if (ok) {
+                float gt[8];  // (P - 1) * 64 <= 8 * kEpiThreads gate totals
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int e = et + j * kEpiThreads;
+                    if (e < (p.P - 1) * 64) gt[j] = __ldcg(p.aggg + (size_t)bh * p.P * 64 + e);
+                }
+                for (int e0 = et; e0 < nA; e0 += 8 * kEpiThreads) {  // one pass: nA <= 8 * kEpiThreads
+                    float2 t[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int e = e0 + j * kEpiThreads, s2 = e / m;
+                        if (e < nA) t[j] = __ldcg(agp + (size_t)s2 * 2048 + u0 + (e - s2 * m));
+                    }
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        if (e0 + j * kEpiThreads < nA) sA[e0 + j * kEpiThreads] = t[j];
+                }
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int e = et + j * kEpiThreads;
+                    if (e < (p.P - 1) * 64) sG[e] = gt[j];
+                }
+            }
+            named_bar_sync(kBarEpi, kEpiThreads);
+            if (ok) {
+                for (int uu = et; uu < m; uu += kEpiThreads) {
+                    const int u = u0 + uu, i = (2 * u) & 63;  // key dim of the pair's first element
                     float2 R = make_float2(0.f, 0.f);
-                    for (int s0 = 0; s0 < p.P - 1; s0 += 8) {
-                        float2 a[8];  // up to eight aggregates in flight
-#pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            if (s0 + e < p.P - 1) a[e] = __ldcg(agp + (size_t)(s0 + e) * 2048 + u);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            if (s0 + e < p.P - 1) {
-                                R = ffma2(ex2_2(ld2(sGt + (s0 + e) * 64 + i)), R, a[e]);
-                                __stcg(sinp + (size_t)(s0 + e + 1) * 2048 + u, R);
-                            }
+                    for (int s2 = 0; s2 < p.P - 1; ++s2) {
+                        R = ffma2(ex2_2(ld2(sG + s2 * 64 + i)), R, sA[s2 * m + uu]);
+                        __stcg(sinp + (size_t)(s2 + 1) * 2048 + u, R);
                     }
                 }
             }
@@ -1080,6 +1115,8 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
     __syncthreads();
     tc_fence_after_sync();
     if (warp == kWarpMma) tmem_dealloc(tbase, kTmemCols);
+    // coop: more arrivals than CTAs means the header was not zero at launch
+    if (tid == 0 && p.coop && arrival >= (unsigned)(p.BH * p.P)) latch_error(p.err, kDevErrWorkspace);
     if (tid == 0) {
         __threadfence();
         const unsigned prev = atomicAdd(&p.ctr[1], 1u);
@@ -1126,7 +1163,7 @@ Plan make_plan(const Problem &pr) {
     const int pmax = nc < kMaxSegments ? nc : kMaxSegments;
     for (int P = 2; P <= pmax; ++P) {
         if ((long long)bh * P > kWsMaxFlags) break;
-        if ((long long)bh * P <= kSMs && bh * P <= kWsMaxFlags / 2) {
+        if ((long long)bh * P <= kSMs && bh * P <= kWsMaxFlags / 2 && P <= kMaxScanSegments) {
             // one wave: the cost falls with L while the last segment is the
             // longest and rises after, so floor and ceil of nc / P bracket it
             for (int L = nc / P; L <= (nc + P - 1) / P; ++L) {

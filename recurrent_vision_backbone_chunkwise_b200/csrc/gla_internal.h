@@ -49,6 +49,10 @@ int ensure_smem(const void *func, size_t bytes);
 int encode_tile_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int rank,
                     const uint64_t *dims, const uint64_t *strides, const uint32_t *box,
                     bool swizzle128);
+// The same with the shared-memory swizzle span in bytes (0, 32, 64 or 128).
+int encode_tile_map_sw(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int rank,
+                       const uint64_t *dims, const uint64_t *strides, const uint32_t *box,
+                       int swizzle_bytes);
 
 // Single-kernel tensor-core path (gla_fused.cu): fp16/bf16, chunk 64, d_k and d_v
 // each 64 or 128 (head sizes of 128 as one launch per 64-wide part).
@@ -64,6 +68,12 @@ int error_word(int **out);
 // Three-phase CUDA-core path (gla_generic.cu): all dtypes, chunk 32 or 64.
 size_t generic_workspace_bytes(const Problem &p);
 int launch_generic(const Problem &p, void *ws, cudaStream_t st);
+
+// The library's tensor-core GEMM after its argument checks (tc_gemm.cu):
+// out[M, N] = in[M, K] . W[N, K]^T (+ bias[N]) (+ resid[M, N]), row-major fp16
+// or bf16, N and K multiples of 8, resid may be out.
+int dense_gemm(int dtype, long long M, int N, int K, const void *in, const void *w, const void *bias,
+               const void *resid, void *out, cudaStream_t st);
 
 // Spatial SwiGLU block after its argument checks (swiglu.cu), with an optional
 // residual: y = resid + SwiGLU(x) (resid and y may be the same tensor).  The

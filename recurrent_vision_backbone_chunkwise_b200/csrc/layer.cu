@@ -14,7 +14,6 @@
 #include "gla_common.cuh"
 #include "gla_internal.h"
 #include "io_pack.cuh"
-#include "lt_gemm.h"
 
 namespace gtr {
 namespace {
@@ -158,7 +157,7 @@ Layout layout(int B, int gh, int gw, int C, int F, int dtype) {
     l.sw_bytes = gtr_swiglu_workspace_size(B, gh, gw, C, F, dtype);
     l.gla = up(l.t + act);
     l.sw = up(l.gla + l.gla_bytes);
-    l.total = up(l.sw + l.sw_bytes);  // the swiglu workspace ends with a cuBLASLt scratch area
+    l.total = up(l.sw + l.sw_bytes);
     return l;
 }
 
@@ -186,8 +185,6 @@ int layer_norm(const T *x, const float *w, const float *b, T *y, long long M, in
 template <typename T>
 int layer_impl(T *x, const GtrLayerWeights *w, int B, int gh, int gw, int C, int F, int dir, int dtype, char *ws,
                const Layout &l, cudaStream_t st) {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return GTR_GLA_ERR_CUDA;
     const long long M = (long long)B * gh * gw, N = (long long)gh * gw;
     const int H = C / 64;
     T *x1 = reinterpret_cast<T *>(ws + l.x1), *P = reinterpret_cast<T *>(ws + l.P);
@@ -195,11 +192,10 @@ int layer_impl(T *x, const GtrLayerWeights *w, int B, int gh, int gw, int C, int
     T *v = reinterpret_cast<T *>(ws + l.v), *z = reinterpret_cast<T *>(ws + l.z);
     T *t = reinterpret_cast<T *>(ws + l.t);
     float *la = reinterpret_cast<float *>(ws + l.la);
-    void *lt_ws = ws + l.sw + (l.sw_bytes - kLtWorkspace);  // the SwiGLU scratch tail, free between its calls
     int rc;
     // token mixer
     if ((rc = layer_norm<T>(x, w->ln1_w, w->ln1_b, x1, M, C, st))) return rc;
-    if ((rc = lt_gemm(dev, dtype, M, 5 * C, C, x1, w->w_proj, nullptr, nullptr, P, lt_ws, st))) return rc;
+    if ((rc = dense_gemm(dtype, M, 5 * C, C, x1, w->w_proj, nullptr, nullptr, P, st))) return rc;
     split_heads_kernel<T><<<grid_for(M * 5 * C / 8, 256), 256, 0, st>>>(P, w->b_a, q, k, v, la, z, M, N, C);
     note_launch();
     if (cudaPeekAtLastError() != cudaSuccess) return GTR_GLA_ERR_CUDA;
@@ -207,7 +203,7 @@ int layer_impl(T *x, const GtrLayerWeights *w, int B, int gh, int gw, int C, int
     if ((rc = gtr_gla_fwd_tail(q, k, v, la, z, w->w_n, kTailEps, t, nullptr, B, H, gh, gw, 64, 64, dir, dtype,
                                ws + l.gla, l.gla_bytes, st)))
         return rc;
-    if ((rc = lt_gemm(dev, dtype, M, C, C, t, w->w_o, nullptr, x, x, lt_ws, st))) return rc;
+    if ((rc = dense_gemm(dtype, M, C, C, t, w->w_o, nullptr, x, x, st))) return rc;
     // channel mixer
     if ((rc = layer_norm<T>(x, w->ln2_w, w->ln2_b, x1, M, C, st))) return rc;
     return swiglu_apply(x1, w->w_gu, w->b_gu, w->w_dw, w->b_dw, w->w_down, w->b_down, x, x, B, gh, gw, C, F, dtype,

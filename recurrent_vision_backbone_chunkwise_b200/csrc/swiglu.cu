@@ -1,6 +1,6 @@
 // swiglu.cu -- Spatial SwiGLU forward (GTR's channel mixer) on sm_100a:
-// the two dense projections as cuBLASLt GEMMs on the tensor cores, and one
-// kernel of this library between them for everything that is not a GEMM:
+// the two dense projections on the library's tensor-core GEMM (tc_gemm.cu),
+// and one kernel between them for everything that is not a GEMM:
 // the projection biases, the 3 x 3 depthwise convolution of the value branch
 // over the patch grid, the SiLU gate and the product.
 //
@@ -15,7 +15,6 @@
 #include "gla_common.cuh"
 #include "gla_internal.h"
 #include "io_pack.cuh"
-#include "lt_gemm.h"
 #include "sm100.cuh"
 
 namespace gtr {
@@ -277,21 +276,8 @@ __global__ void __launch_bounds__(kDwThreads, 1) swiglu_dw_gate_kernel(
                 latch_error(err, kDevErrTimeout);
 }
 
-// y[m, c] += bias[c] in fp32: the fallback for a cuBLASLt that offers no
-// bias epilogue for this GEMM (on B200 with these types it does, and this
-// kernel does not run).
-template <typename T>
-__global__ void add_bias_kernel(T *y, const float *bias, size_t M, int C) {
-    const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;  // pair index
-    if (i >= M * (size_t)C / 2) return;
-    const int c = (int)((2 * i) % C);
-    uint32_t *p = reinterpret_cast<uint32_t *>(y) + i;
-    const float2 o = Pair<T>::unpack(*p);
-    *p = Pair<T>::pack(o.x + bias[c], o.y + bias[c + 1]);
-}
-
 struct SwLayout {
-    size_t gu, h, bd, lt, total;
+    size_t gu, h, bd, total;
 };
 
 SwLayout sw_layout(long long M, int C, int F, size_t es) {
@@ -300,8 +286,7 @@ SwLayout sw_layout(long long M, int C, int F, size_t es) {
     l.gu = 0;
     l.h = up((size_t)M * 2 * F * es);
     l.bd = up(l.h + (size_t)M * F * es);
-    l.lt = up(l.bd + (size_t)C * es);
-    l.total = l.lt + kLtWorkspace;
+    l.total = up(l.bd + (size_t)C * es);
     return l;
 }
 
@@ -380,41 +365,26 @@ int launch_dw_gate(int dtype, const void *gu, const float *b_gu, const float *w_
 }  // namespace
 
 // The block after argument checks (shared with the backbone layer): y = x +
-// ... when resid = x is given (the down projection adds it as cuBLASLt's C
-// operand; y may be x itself).
+// ... when resid = x is given (the down projection's epilogue adds it; y may
+// be x itself).
 int swiglu_apply(const void *x, const void *w_gu, const float *b_gu, const float *w_dw, const float *b_dw,
                  const void *w_down, const float *b_down, const void *resid, void *y, int B, int grid_h,
                  int grid_w, int C, int F, int dtype, void *workspace, cudaStream_t stream) {
     const long long M = (long long)B * grid_h * grid_w;
     const SwLayout l = sw_layout(M, C, F, 2);
     int rc;
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return GTR_GLA_ERR_CUDA;
     char *ws = static_cast<char *>(workspace);
-    void *gu = ws + l.gu, *h = ws + l.h, *bd = ws + l.bd, *lt_ws = ws + l.lt;
+    void *gu = ws + l.gu, *h = ws + l.h, *bd = ws + l.bd;
     // 1. [g | u] without biases (the kernel adds them in fp32)
-    rc = lt_gemm(dev, dtype, M, 2 * F, C, x, w_gu, nullptr, nullptr, gu, lt_ws, stream);
+    rc = dense_gemm(dtype, M, 2 * F, C, x, w_gu, nullptr, nullptr, gu, stream);
     if (rc) return rc;
     // 2. biases, depthwise 3 x 3 on the value branch, SiLU gate, product
     rc = launch_dw_gate(dtype, gu, b_gu, w_dw, b_dw, h, b_down, bd, B, grid_h, grid_w, F, C, stream);
     if (rc) return rc;
-    // 3. y = h W_d^T + b_d (the bias, copied to the I/O dtype by the kernel
-    //    above, in the GEMM's epilogue; one pass of this library in fp32 if
-    //    cuBLASLt offers no such epilogue)
-    rc = lt_gemm(dev, dtype, M, C, F, h, w_down, bd, resid, y, lt_ws, stream);
-    if (rc) {
-        rc = lt_gemm(dev, dtype, M, C, F, h, w_down, nullptr, resid, y, lt_ws, stream);
-        if (rc) return rc;
-        const size_t pairs = (size_t)M * C / 2;
-        const unsigned blocks = (unsigned)((pairs + 255) / 256);
-        if (dtype == GTR_GLA_BF16)
-            add_bias_kernel<__nv_bfloat16><<<blocks, 256, 0, stream>>>(static_cast<__nv_bfloat16 *>(y), b_down,
-                                                                       (size_t)M, C);
-        else
-            add_bias_kernel<__half><<<blocks, 256, 0, stream>>>(static_cast<__half *>(y), b_down, (size_t)M, C);
-        note_launch();
-        if (cudaPeekAtLastError() != cudaSuccess) return GTR_GLA_ERR_CUDA;
-    }
+    // 3. y = h W_d^T + b_d (+ resid): the bias (copied to the I/O dtype by the
+    //    kernel above) and the residual in the GEMM's epilogue
+    rc = dense_gemm(dtype, M, C, F, h, w_down, bd, resid, y, stream);
+    if (rc) return rc;
     return GTR_GLA_OK;
 }
 

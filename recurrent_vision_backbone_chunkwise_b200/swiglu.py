@@ -1,6 +1,6 @@
 """ctypes binding of the Spatial SwiGLU entry points of libgtr_gla.so
-(argument marshalling only; the arithmetic runs in the library: cuBLASLt for
-the two projections, the library's own kernel for the rest).  See
+(argument marshalling only; the arithmetic runs in the library's kernels: its
+tensor-core GEMM for the two projections, its fused kernel for the rest).  See
 ``include/gtr_swiglu.h`` for the contract.
 
 Tensors are torch CUDA tensors, contiguous: x [B, grid_h, grid_w, C] and the

@@ -26,7 +26,7 @@ def declared_functions():
     for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
         text = open(h).read()
         text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-        for m in re.finditer(r"\b(gtr_(?:gla|swiglu|output_tail|layer|backbone)_\w+)\s*\(", text):
+        for m in re.finditer(r"\b(gtr_(?:gla|swiglu|output_tail|layer|backbone|gemm)_\w+)\s*\(", text):
             names.add(m.group(1))
     return sorted(names)
 
@@ -36,7 +36,7 @@ def test_header_declares_entry_points():
     for n in ("gtr_gla_fwd", "gtr_gla_fwd_ex", "gtr_gla_workspace_size", "gtr_gla_status",
               "gtr_gla_strerror", "gtr_gla_release", "gtr_gla_launch_count",
               "gtr_swiglu_fwd", "gtr_swiglu_workspace_size", "gtr_output_tail_fwd",
-              "gtr_layer_fwd", "gtr_backbone_fwd", "gtr_layer_workspace_size"):
+              "gtr_layer_fwd", "gtr_backbone_fwd", "gtr_layer_workspace_size", "gtr_gemm_fwd"):
         assert n in names
 
 
@@ -45,10 +45,11 @@ def test_library_exports_every_declared_symbol(gla):
     for n in declared_functions():
         assert hasattr(lib, n), f"{n} declared in include/ but not exported"
         # the binding forwards under the same name
-        from recurrent_vision_backbone_chunkwise_b200 import layer, output_tail, swiglu
+        from recurrent_vision_backbone_chunkwise_b200 import gemm, layer, output_tail, swiglu
 
         mod = (swiglu if n.startswith("gtr_swiglu_") else output_tail if n.startswith("gtr_output_tail_")
-               else layer if n.startswith(("gtr_layer_", "gtr_backbone_")) else gla)
+               else layer if n.startswith(("gtr_layer_", "gtr_backbone_"))
+               else gemm if n.startswith("gtr_gemm_") else gla)
         assert hasattr(mod, n), n
 
 
@@ -311,3 +312,18 @@ def test_checked_build_exports_every_declared_symbol(gla):
         assert hasattr(lib, n), n
     lib.gtr_gla_strerror.restype = ctypes.c_char_p
     assert b"index check" in lib.gtr_gla_strerror(-13)
+
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(x=0), -1), (dict(w=0), -1), (dict(out=0), -1), (dict(M=0), -2), (dict(N=12), -2), (dict(K=20), -2),
+    (dict(dtype=2), -6), (dict(x=0x20000004), -5), (dict(bias=0x60000002), -5),
+    (dict(out=0x20000000 + 64), -11), (dict(resid=0x70000000 + 128), -11),
+])
+def test_gemm_argument_errors(gla, kw, code):
+    a = dict(x=0x20000000, w=0x40000000, bias=0x60000000, resid=0, out=0x70000000, M=100, N=64, K=64,
+             dtype=gla.F16)
+    a.update(kw)
+    vp = ctypes.c_void_p
+    assert gla._lib.gtr_gemm_fwd(vp(a["x"]), vp(a["w"]), vp(a["bias"]), vp(a["resid"]), vp(a["out"]),
+                                 ctypes.c_longlong(a["M"]), a["N"], a["K"], a["dtype"], None) == code
