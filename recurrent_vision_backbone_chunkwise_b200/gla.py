@@ -227,3 +227,36 @@ def gtr_gla_fwd_tail(q, k, v, log_alpha, z, w_n, direction, eps=1e-5, y=None, fi
     if rc != 0:
         raise GlaError(rc)
     return y, final_state
+
+
+_lib.gtr_gla_bwd.argtypes = [_vp] * 10 + [_int] * 8 + [_vp, _sz, _vp]
+_lib.gtr_gla_bwd.restype = _int
+_lib.gtr_gla_bwd_workspace_size.argtypes = [_int] * 6
+_lib.gtr_gla_bwd_workspace_size.restype = _sz
+
+
+def gtr_gla_bwd_workspace_size(B, H, grid_h, grid_w, d_k=64, d_v=64) -> int:
+    return int(_lib.gtr_gla_bwd_workspace_size(B, H, grid_h, grid_w, d_k, d_v))
+
+
+def gtr_gla_bwd(q, k, v, log_alpha, d_out, direction, d_final_state=None, workspace=None, stream=None):
+    """Gradients (dq, dk, dv, dlog_alpha) of sum(d_out * out) + sum(d_final_state *
+    final_state) for the forward pass with the same arguments; see
+    ``include/gtr_gla_bwd.h``.  dq, dk, dv in q's dtype, dlog_alpha fp32."""
+    _validate(q, k, v, log_alpha, d_out, d_final_state)
+    B, H, gh, gw, dk_, dv_ = _shape(q, v)
+    dtype = _DTYPE_CODE.get(q.dtype)
+    if dtype is None:
+        raise ValueError(f"unsupported dtype {q.dtype}")
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dla = torch.empty_like(log_alpha)
+    need = gtr_gla_bwd_workspace_size(B, H, gh, gw, dk_, dv_)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    _check("workspace", workspace, (workspace.numel(),), torch.uint8, q.device)
+    rc = _lib.gtr_gla_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(d_out), _ptr(d_final_state),
+                          _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dla), B, H, gh, gw, dk_, dv_, int(direction), dtype,
+                          _ptr(workspace), workspace.numel(), _vp(_stream_handle(stream)))
+    if rc != 0:
+        raise GlaError(rc)
+    return dq, dk, dv, dla

@@ -327,3 +327,28 @@ def test_gemm_argument_errors(gla, kw, code):
     vp = ctypes.c_void_p
     assert gla._lib.gtr_gemm_fwd(vp(a["x"]), vp(a["w"]), vp(a["bias"]), vp(a["resid"]), vp(a["out"]),
                                  ctypes.c_longlong(a["M"]), a["N"], a["K"], a["dtype"], None) == code
+
+
+# ---------------------------------------------------------------- backward pass
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=0), -1), (dict(dla=0), -1), (dict(B=0), -2), (dict(dk=128), -3), (dict(dir=4), -4),
+    (dict(dq=Q + 8), -5), (dict(dtype=3), -6), (dict(ws=0), -8), (dict(wsb=16), -8),
+    (dict(dq=K), -11), (dict(dv=0xA0000000 + 256), -11), (dict(dla=LA), -11),
+])
+def test_backward_argument_errors(gla, kw, code):
+    a = dict(q=Q, k=K, v=V, la=LA, dO=OUT, dsf=FS, dq=0xA0000000, dk=0xB0000000, dv=0xC0000000,
+             dla=0xD0000000, B=1, H=2, gh=4, gw=4, dk_=64, dv_=64, dir=0, dtype=gla.F16, ws=WS, wsb=1 << 30)
+    if "dk" in kw and isinstance(kw["dk"], int) and kw["dk"] == 128:
+        kw = dict(dk_=128)
+    a.update(kw)
+    vp = ctypes.c_void_p
+    assert gla._lib.gtr_gla_bwd(vp(a["q"]), vp(a["k"]), vp(a["v"]), vp(a["la"]), vp(a["dO"]), vp(a["dsf"]),
+                                vp(a["dq"]), vp(a["dk"]), vp(a["dv"]), vp(a["dla"]), a["B"], a["H"], a["gh"],
+                                a["gw"], a["dk_"], a["dv_"], a["dir"], a["dtype"], vp(a["ws"]), a["wsb"],
+                                None) == code
+
+
+def test_backward_workspace_size(gla):
+    assert gla.gtr_gla_bwd_workspace_size(1, 6, 40, 40) > 0
+    assert gla.gtr_gla_bwd_workspace_size(1, 6, 40, 40, 128, 128) == 0
