@@ -385,6 +385,111 @@ def run_backbone(args):
         dist.destroy_process_group()
 
 
+def run_bwd(args):
+    """Backward leg (not the headline): the gradients of the attention on the
+    workload (d = 64, chunk 64), image tokens/s per call (one direction per
+    call, the four cycled) and its HBM roofline fraction: per token-head q, k,
+    v, d_out read and dq, dk, dv written at 2 d bytes each, log_alpha read and
+    dlog_alpha written at 4 d bytes each (1536 B at d = 64), plus the final-state
+    gradient; the fp64 oracle on the host."""
+    import torch
+    from recurrent_vision_backbone_chunkwise_b200 import gla
+
+    ri = rank_info()
+    torch.cuda.set_device(ri.local_rank)
+    dev = torch.device("cuda", ri.local_rank)
+    dist = dist_setup(ri, dev)
+    shape, dtype = CONFIGS[args.config]
+    dtype = "f16" if dtype == "f32" else dtype
+    if shape.d_k != 64 or shape.d_v != 64:
+        raise SystemExit("the backward pass takes head size 64")
+    B, H, gh, gw = shape.B, shape.H, shape.grid_h, shape.grid_w
+    host = make_inputs(shape, dtype, seed=replica_seed(0, ri.rank))
+    g = torch.Generator().manual_seed(replica_seed(7, ri.rank))
+    hdo = torch.randn(host[2].shape, generator=g).to(host[2].dtype)
+    hdsf = torch.randn(B, H, 64, 64, generator=g)
+    units = B * H * gh * gw
+    call_bytes = 1536 * units + B * H * 64 * 64 * 4
+    R = max(2, math.ceil(2 * L2_BYTES / call_bytes))
+    sets = [[t.to(dev) for t in (*host, hdo, hdsf)] for _ in range(R)]
+    ws = torch.empty(gla.gtr_gla_bwd_workspace_size(B, H, gh, gw), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(i, ev=None):
+        q, k, v, la, do, dsf = sets[i % R]
+        if ev is not None:
+            ev[0].record(stream)
+        gla.gtr_gla_bwd(q, k, v, la, do, i % 4, d_final_state=dsf, workspace=ws, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            step(i)
+    stream.synchronize()
+    assert gla.gtr_gla_status(stream) == 0
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)] for _ in range(K)]
+    launches0 = gla.gtr_gla_launch_count()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(K):
+            step(i, evs[i])
+    launches = gla.gtr_gla_launch_count() - launches0
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(smi_index(ri.local_rank))
+    sampler.start()
+    time.sleep(0.2)
+    dist_barrier(dist)
+    torch.cuda.synchronize()
+    t0 = time.time()
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        graph.replay()
+        end.record(stream)
+    torch.cuda.synchronize()
+    t1 = time.time()
+    dist_barrier(dist)
+    clocks = sampler.stop(t0, t1)
+    assert gla.gtr_gla_status(stream) == 0
+    elapsed = max_over_ranks(start.elapsed_time(end), device=dev)
+    call_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    del graph
+    mean_s = statistics.mean(call_ms) / 1000.0
+    peak, kind = measured_peaks()
+    src = "measured copy bandwidth (burst)" if kind == "measured" else "fallback (6.65 TB/s)"
+    achieved = call_bytes / mean_s / 1e9
+    line = {
+        "metric": "GLA backward image tokens/s and us per call; % of HBM roofline", "value":
+            aggregate_rate(ri.world, K, B * gh * gw, elapsed), "unit": "tokens/s", "n_gpus": ri.world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": elapsed / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": dtype, "data": "synthetic",
+        "config": {"workload": f"bwd_{args.config}", "B": B, "H": H, "grid": [gh, gw], "d": 64, "chunk": 64,
+                   "directions": 4, "l2": f"inputs rotate over {R} sets", "cuda_graph": True},
+        "kernel_us_per_call": {"mean": 1e6 * mean_s, "median": 1e3 * statistics.median(call_ms),
+                               "min": 1e3 * min(call_ms)},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": None, "peak_source": src, "bytes_per_call": call_bytes,
+                     "timed_unit": "one gtr_gla_bwd call (its seven kernels)"},
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+    }
+    if ri.rank == 0 and ri.world == 1 and not args.no_cpu_baseline:
+        import oracle.backward as ob
+
+        reps, t0 = 0, time.perf_counter()
+        while time.perf_counter() - t0 < 10.0 and reps < 100:
+            ob.backward(*host, hdo, reps % 4, d_final_state=hdsf)
+            reps += 1
+        el = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": reps * B * gh * gw / el, "unit": "tokens/s", "cores": host_threads(),
+                                "kind": "oracle", "sample": f"{reps} full backward calls (fp64) in {el:.1f} s"}
+    if ri.rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
 def run_tail(args):
     """Output-tail leg (not the headline): token-heads/s of the tail on the
     workload's attention output (B, H, grid, d_v), its HBM roofline fraction
@@ -832,9 +937,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-config", action="store_true",
                     help="time only --config (skip the other token counts of the metric)")
-    ap.add_argument("--op", default="gla", choices=["gla", "swiglu", "tail", "backbone"],
+    ap.add_argument("--op", default="gla", choices=["gla", "swiglu", "tail", "backbone", "bwd"],
                     help="gla: the headline (chunkwise GLA); swiglu: the Spatial SwiGLU block; "
-                         "tail: the attention's output tail; backbone: the 12-layer stack")
+                         "tail: the attention's output tail; backbone: the 12-layer stack; "
+                         "bwd: the attention's backward pass")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.op == "swiglu" and args.impl == "ours":
@@ -845,6 +951,9 @@ def main():
         return
     if args.op == "backbone" and args.impl == "ours":
         run_backbone(args)
+        return
+    if args.op == "bwd" and args.impl == "ours":
+        run_bwd(args)
         return
 
     if args.impl == "reference":

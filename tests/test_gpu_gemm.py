@@ -34,6 +34,8 @@ def rel(a, b):
     (1000, 136, 72, True, False, torch.float16),      # ragged M, N and K tails
     (1, 8, 8, True, True, torch.float16),             # one row
     (3333, 512, 256, False, True, torch.bfloat16),
+    (300, 256, 1000, True, True, torch.float16),      # K not a multiple of 64 (the last block zero-filled)
+    (1600, 768, 3072, False, False, torch.bfloat16),  # long K
 ])
 def test_gemm_matches_float64(M, N, K, bias, resid, dtype):
     from recurrent_vision_backbone_chunkwise_b200 import gemm, gla
@@ -61,3 +63,17 @@ def test_gemm_accumulates_in_place():
     gemm.gtr_gemm_fwd(x.cuda(), w.cuda(), resid=out, out=out)
     assert gla.gtr_gla_status() == 0
     assert rel(out, ref(x, w, None, r)) <= TOL[torch.float16]
+
+
+def test_gemm_is_deterministic():
+    """Fixed accumulation order: two calls agree bit for bit."""
+    from recurrent_vision_backbone_chunkwise_b200 import gemm, gla
+
+    g = torch.Generator().manual_seed(3)
+    x = torch.randn(1600, 1536, generator=g).half().cuda()
+    w = (torch.randn(384, 1536, generator=g) / 40).half().cuda()
+    a = gemm.gtr_gemm_fwd(x, w)
+    b = gemm.gtr_gemm_fwd(x, w)
+    torch.cuda.synchronize()
+    assert gla.gtr_gla_status() == 0
+    assert torch.equal(a, b)
