@@ -80,6 +80,8 @@ def test_fused_edge_grids(lib, grid, direction):
     (Shape(1, 12, 64, 64, 64, 64), "bf16", 3),
     (Shape(1, 2, 20, 24, 128, 128), "f16", 0),  # head size 128 in four parts
     (Shape(1, 2, 20, 24, 64, 128), "f16", 3),
+    (Shape(3, 16, 24, 40, 64, 64), "f16", 0),   # 48 planes x 3 segments of uneven length
+    (Shape(3, 16, 24, 40, 64, 64), "bf16", 3),
 ])
 def test_fused_plans_and_head_sizes(lib, shape, dtype, direction):
     run(lib, shape, dtype, direction, seed=9)

@@ -148,3 +148,117 @@ def test_segments_by_launch_index_can_starve():
         err, hdr, _ = run_launch(1, 4, 1, seed, by_launch_index=True, wait_limit=0.1)
         starved = starved or ("timeout" in err.all)
     assert starved
+
+
+# ------------------------------------------------ the transposed boundary scan
+#
+# One-wave plans run as a cooperative launch (every CTA resident) and
+# exchange boundary states in two rounds (csrc/gla_fused.cu):
+# - every segment but the last publishes its aggregate A_s and gate totals g_s
+#   and raises flag1;
+# - each CTA waits (bounded) for all flag1 of its plane, takes the slice
+#   [seg * npairs / P, (seg + 1) * npairs / P) of the state's element pairs,
+#   runs S_in(s + 1) = diag(e^{g_s}) S_in(s) + A_s over all segments for that
+#   slice, writes that slice of every S_in and raises flag2;
+# - every segment but the first waits (bounded) for all flag2 of its plane and
+#   reads its S_in, which all CTAs of the plane wrote;
+# - the arrival count is checked at the end (a dirty header is reported).
+# The model carries real numbers (d_k x d_v = 4 x 4, 8 pairs) and checks every
+# S_in against the sequential definition, S_in(s) = sum_{t < s}
+# diag(e^{g_{t+1} + ... + g_{s-1}}) A_t.
+
+import numpy as np  # noqa: E402
+
+
+def run_coop_scan(BH, P, seed, *, resident=None, drop_flag2_of=None, dirty_arrivals=0, wait_limit=2.0,
+                  dk=4, dv=4):
+    rng = np.random.default_rng(seed)
+    prng = random.Random(seed)
+    G = BH * P
+    npairs = dk * dv // 2
+    A = rng.standard_normal((BH, P, dk, dv))
+    g = -np.abs(rng.standard_normal((BH, P, dk)))  # log-gate totals, <= 0
+    sin = np.full((BH, P, dk * dv), np.nan)
+    got = np.full((BH, P, dk * dv), np.nan)
+    flag1 = [threading.Event() for _ in range(G)]
+    flag2 = [threading.Event() for _ in range(G)]
+    arrivals = [dirty_arrivals]
+    lock = threading.Lock()
+    err = Errors()
+    sem = threading.Semaphore(resident if resident is not None else G)
+    delays = [prng.uniform(0, 2e-3) for _ in range(G)]
+
+    def cta(block):
+        with sem:
+            with lock:
+                arrival = arrivals[0]
+                arrivals[0] += 1
+            bh, seg = divmod(block, P)  # every CTA resident: the block index names the segment
+            time.sleep(delays[block])  # the pre-pass
+            if seg < P - 1:
+                flag1[bh * P + seg].set()
+            ok = all(flag1[bh * P + j].wait(timeout=wait_limit) for j in range(P - 1))
+            if not ok:
+                err.latch("timeout")
+            else:
+                u0, u1 = seg * npairs // P, (seg + 1) * npairs // P
+                for u in range(u0, u1):
+                    e = np.array([2 * u, 2 * u + 1])
+                    i = e // dv  # key dim of each element
+                    R = np.zeros(2)
+                    for s2 in range(P - 1):
+                        R = np.exp(g[bh, s2, i]) * R + A[bh, s2].reshape(-1)[e]
+                        sin[bh, s2 + 1, e] = R
+            if block != drop_flag2_of and ok:
+                flag2[bh * P + seg].set()
+            if seg > 0:
+                if all(flag2[bh * P + j].wait(timeout=wait_limit) for j in range(P)):
+                    got[bh, seg] = sin[bh, seg]
+                else:
+                    err.latch("timeout")
+            if arrival >= G:  # checked at the end, off the critical path
+                err.latch("workspace_state")
+
+    threads = [threading.Thread(target=cta, args=(b,)) for b in prng.sample(range(G), G)]
+    t0 = time.time()
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join(timeout=60)
+    assert not any(t.is_alive() for t in threads), "a modelled CTA never finished"
+    # the definition, segment by segment
+    ref = np.zeros((BH, P, dk * dv))
+    for bh in range(BH):
+        for s in range(1, P):
+            acc = np.zeros((dk, dv))
+            for t in range(s):
+                acc += np.exp(g[bh, t + 1:s].sum(axis=0))[:, None] * A[bh, t]
+            ref[bh, s] = acc.reshape(-1)
+    return err, got, ref, time.time() - t0
+
+
+@pytest.mark.parametrize("BH,P", [(1, 2), (6, 24), (48, 3), (12, 12), (2, 33)])
+@pytest.mark.parametrize("seed", [0, 1])
+def test_coop_scan_gives_every_segment_its_incoming_state(BH, P, seed):
+    err, got, ref, _ = run_coop_scan(BH, P, seed, wait_limit=5.0)
+    assert err.first is None, err.all
+    np.testing.assert_allclose(got[:, 1:], ref[:, 1:], rtol=1e-12, atol=1e-12)
+
+
+def test_coop_scan_dropped_flag2_times_out_and_ends():
+    err, _, _, wall = run_coop_scan(2, 6, 5, drop_flag2_of=3, wait_limit=0.3)
+    assert err.first == "timeout"
+    assert wall < 10.0
+
+
+def test_coop_scan_reports_a_dirty_arrival_count():
+    err, got, ref, _ = run_coop_scan(1, 4, 6, dirty_arrivals=2, wait_limit=2.0)
+    assert "workspace_state" in err.all
+
+
+def test_coop_scan_needs_every_cta_resident():
+    """Control: with fewer resident CTAs than segments of a plane, a CTA waits
+    for the flag1 of a segment whose CTA cannot start: only the bounded wait
+    ends the run.  This is why the scan runs under a cooperative launch."""
+    err, _, _, _ = run_coop_scan(1, 6, 7, resident=3, wait_limit=0.2)
+    assert "timeout" in err.all
