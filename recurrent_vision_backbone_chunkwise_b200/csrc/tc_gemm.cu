@@ -5,7 +5,8 @@
 // and residual added in fp32, one rounding (see include/gtr_gemm.h).
 //
 // Persistent CTAs (at most one per SM) walk output tiles of 128 rows x BN
-// columns (BN = 256, or 128 when 256-wide tiles would leave SMs idle).  Per
+// columns (BN = 256, 128 or 64: the fewest waves of tiles, weighted by the
+// operand bytes a tile reads).  Per
 // tile, K runs in blocks of 64 through a 4-stage shared-memory ring filled by
 // TMA (both operands K-major with the 128-byte swizzle) and drained by
 // tcgen05.mma M128 x BN x K16 into one of two TMEM accumulators.  Four
@@ -286,16 +287,22 @@ int dense_gemm(int dtype, long long M, int N, int K, const void *in, const void 
     p.num_m = (int)((M + GM - 1) / GM);
     int rc = error_word(&p.err);
     if (rc) return rc;
-    // tile width: the fewer waves of tiles, weighted by the tile's width plus
-    // a fixed cost per tile (256 when equal)
+    // tile width (256, 128 or 64 columns): the fewest waves of tiles, each
+    // weighted by the operand rows it reads (128 + BN), its MMA work (BN) and a
+    // fixed cost (measured on B200: this picks 128 for 1600 x 3072 x 384, 64
+    // for 1600 x 384 x 1536, 256 for 12800 x 6144 x 768)
     auto cost = [&](long long bn) {
         const long long tiles = (long long)p.num_m * ((N + bn - 1) / bn);
-        return ((tiles + sms - 1) / sms) * (bn + 64);
+        return ((tiles + sms - 1) / sms) * (GM + 2 * bn + 64);
     };
-    const bool wide = cost(256) <= cost(128);
+    const int bn = cost(256) <= cost(128) ? (cost(256) <= cost(64) ? 256 : 64) : (cost(128) <= cost(64) ? 128 : 64);
     if (dtype == GTR_GLA_BF16)
-        return wide ? launch<__nv_bfloat16, 256>(p, in, w, sms, st) : launch<__nv_bfloat16, 128>(p, in, w, sms, st);
-    return wide ? launch<__half, 256>(p, in, w, sms, st) : launch<__half, 128>(p, in, w, sms, st);
+        return bn == 256   ? launch<__nv_bfloat16, 256>(p, in, w, sms, st)
+               : bn == 128 ? launch<__nv_bfloat16, 128>(p, in, w, sms, st)
+                           : launch<__nv_bfloat16, 64>(p, in, w, sms, st);
+    return bn == 256 ? launch<__half, 256>(p, in, w, sms, st)
+           : bn == 128 ? launch<__half, 128>(p, in, w, sms, st)
+                       : launch<__half, 64>(p, in, w, sms, st);
 }
 
 }  // namespace gtr
