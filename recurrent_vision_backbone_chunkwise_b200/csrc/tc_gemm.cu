@@ -5,8 +5,8 @@
 // and residual added in fp32, one rounding (see include/gtr_gemm.h).
 //
 // Persistent CTAs (at most one per SM) walk output tiles of 128 rows x BN
-// columns (BN = 256, 128 or 64: the fewest waves of tiles, weighted by the
-// operand bytes a tile reads).  Per
+// columns (BN = 256, 192, 128 or 64: the fewest waves of tiles, weighted by
+// the operand bytes and MMA work of a tile).  Per
 // tile, K runs in blocks of 64 through a 4-stage shared-memory ring filled by
 // TMA (both operands K-major with the 128-byte swizzle) and drained by
 // tcgen05.mma M128 x BN x K16 into one of two TMEM accumulators.  Four
@@ -43,7 +43,8 @@ template <int BN> struct GemmCfg {
     static constexpr uint32_t kStage = kGABytes + BN * GK * 2;
     static constexpr uint32_t kOffOut = kGStages * kStage;  // 4 warps x 2 output staging buffers
     static constexpr uint32_t kSmem = kOffOut + 8 * kOutChunk + 1024;  // + alignment slack
-    static constexpr uint32_t kTmemCols = 2 * BN;                      // two accumulators
+    // two accumulators (at columns 0 and BN), allocated as a power of two
+    static constexpr uint32_t kTmemCols = 2 * BN <= 128 ? 128 : 2 * BN <= 256 ? 256 : 512;
 };
 static_assert(GemmCfg<256>::kSmem <= 232448, "shared memory");
 
@@ -287,22 +288,32 @@ int dense_gemm(int dtype, long long M, int N, int K, const void *in, const void 
     p.num_m = (int)((M + GM - 1) / GM);
     int rc = error_word(&p.err);
     if (rc) return rc;
-    // tile width (256, 128 or 64 columns): the fewest waves of tiles, each
-    // weighted by the operand rows it reads (128 + BN), its MMA work (BN) and a
-    // fixed cost (measured on B200: this picks 128 for 1600 x 3072 x 384, 64
-    // for 1600 x 384 x 1536, 256 for 12800 x 6144 x 768)
+    // tile width (256, 192, 128 or 64 columns): the fewest waves of tiles,
+    // each weighted by the operand rows it reads (128 + BN), its MMA work (BN)
+    // and a fixed cost (measured on B200: this picks 128 for 1600 x 3072 x 384,
+    // 64 for 1600 x 384 x 1536, 256 for 12800 x 6144 x 768, 192 for
+    // 12800 x 768 x 3072)
     auto cost = [&](long long bn) {
         const long long tiles = (long long)p.num_m * ((N + bn - 1) / bn);
         return ((tiles + sms - 1) / sms) * (GM + 2 * bn + 64);
     };
-    const int bn = cost(256) <= cost(128) ? (cost(256) <= cost(64) ? 256 : 64) : (cost(128) <= cost(64) ? 128 : 64);
-    if (dtype == GTR_GLA_BF16)
-        return bn == 256   ? launch<__nv_bfloat16, 256>(p, in, w, sms, st)
-               : bn == 128 ? launch<__nv_bfloat16, 128>(p, in, w, sms, st)
-                           : launch<__nv_bfloat16, 64>(p, in, w, sms, st);
-    return bn == 256 ? launch<__half, 256>(p, in, w, sms, st)
-           : bn == 128 ? launch<__half, 128>(p, in, w, sms, st)
-                       : launch<__half, 64>(p, in, w, sms, st);
+    int bn = 256;
+    for (int c : {192, 128, 64})
+        if (cost(c) < cost(bn)) bn = c;
+    if (dtype == GTR_GLA_BF16) {
+        switch (bn) {
+            case 256: return launch<__nv_bfloat16, 256>(p, in, w, sms, st);
+            case 192: return launch<__nv_bfloat16, 192>(p, in, w, sms, st);
+            case 128: return launch<__nv_bfloat16, 128>(p, in, w, sms, st);
+            default: return launch<__nv_bfloat16, 64>(p, in, w, sms, st);
+        }
+    }
+    switch (bn) {
+        case 256: return launch<__half, 256>(p, in, w, sms, st);
+        case 192: return launch<__half, 192>(p, in, w, sms, st);
+        case 128: return launch<__half, 128>(p, in, w, sms, st);
+        default: return launch<__half, 64>(p, in, w, sms, st);
+    }
 }
 
 }  // namespace gtr

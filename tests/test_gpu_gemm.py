@@ -36,6 +36,8 @@ def rel(a, b):
     (3333, 512, 256, False, True, torch.bfloat16),
     (300, 256, 1000, True, True, torch.float16),      # K not a multiple of 64 (the last block zero-filled)
     (1600, 768, 3072, False, False, torch.bfloat16),  # long K
+    (3840, 768, 512, True, True, torch.float16),      # 192-wide tiles
+    (3840, 760, 256, False, True, torch.bfloat16),    # 192-wide tiles with a column tail
 ])
 def test_gemm_matches_float64(M, N, K, bias, resid, dtype):
     from recurrent_vision_backbone_chunkwise_b200 import gemm, gla
