@@ -49,6 +49,7 @@
 // Chunks whose in-chunk gate span exceeds kSpanLimit (e^{-b} would leave fp32
 // range) get their scores from an exact CUDA-core evaluation by the operand
 // warps (every factor <= 1), stored straight into TMEM.
+#include <algorithm>
 #include <cstring>
 #include <map>
 #include <mutex>
@@ -142,6 +143,10 @@ struct FusedParams {
     // boundary states come from the transposed scan; otherwise each segment
     // folds the earlier aggregates itself
     int coop;
+    // the segment that holds the chunks left over, nc - (P - 1) L of them:
+    // the last (0) or the first (1; it starts its main pass without waiting
+    // for the scan's second round, its incoming state being zero)
+    int rem_first;
     // Head sizes of 128 run as 64-wide sub-problems (every key row of the
     // state evolves on its own and every value column too; the output is
     // the sum over the key halves): `out` and `final_state` point at the
@@ -334,8 +339,12 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
     const uint32_t tbase = s_tmem;
     const int ticket = s_ticket;
     const int bh = ticket / p.P, seg = ticket % p.P;
-    // segments 0 .. P-2 have L chunks, the last one the rest (which may be longer)
-    const int c_begin = seg * p.L, c_end = (seg == p.P - 1) ? p.nc : min(c_begin + p.L, p.nc);
+    // every segment has L chunks but one, which has the rest (possibly more):
+    // the last, or with rem_first the first
+    const int rem = p.nc - (p.P - 1) * p.L;
+    const int c_begin = p.rem_first ? (seg == 0 ? 0 : rem + (seg - 1) * p.L) : seg * p.L;
+    const int c_end = p.rem_first ? (seg == 0 ? rem : c_begin + p.L)
+                                  : ((seg == p.P - 1) ? p.nc : min(c_begin + p.L, p.nc));
     const int L = c_end - c_begin;
     const int npre = (seg < p.P - 1) ? L : 0;  // the last segment needs no aggregate
     const int n_items = npre + L;
@@ -1140,7 +1149,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
 constexpr int kSMs = 148;
 
 struct Plan {
-    int nc, P, L, coop;
+    int nc, P, L, coop, rem_first;
 };
 
 // Segments per (b,h).  More segments put more SMs to work and shorten each
@@ -1155,10 +1164,12 @@ struct Plan {
 // aggregate, the transposed scan, and the fixed cost of publishing and
 // waiting for flags.
 Plan make_plan(const Problem &pr) {
-    constexpr double kMain = 2.2, kPre = 1.2, kFold = 0.5, kFlag = 3.0, kScan = 3.0;
+    // kFlag: publishing and the flag round of the fold; the cooperative plans
+    // split it into the aggregates' round (kFlag1) and the scan's (kFlag2)
+    constexpr double kMain = 2.2, kPre = 1.2, kFold = 0.5, kFlag = 3.0, kScan = 3.0, kFlag1 = 2.0, kFlag2 = 1.8;
     const int nc = (pr.n + FC - 1) / FC;
     const int bh = pr.B * pr.H;
-    Plan best{nc, 1, nc, 0};
+    Plan best{nc, 1, nc, 0, 0};
     double tbest = nc * kMain * (double)((bh + kSMs - 1) / kSMs);
     const int pmax = nc < kMaxSegments ? nc : kMaxSegments;
     for (int P = 2; P <= pmax; ++P) {
@@ -1167,12 +1178,23 @@ Plan make_plan(const Problem &pr) {
             // one wave: the cost falls with L while the last segment is the
             // longest and rises after, so floor and ceil of nc / P bracket it
             for (int L = nc / P; L <= (nc + P - 1) / P; ++L) {
-                const int last = nc - (P - 1) * L;
-                if (L < 1 || last < 1) continue;
-                const double t = L * kPre + kFlag + kScan + (last > L ? last : L) * kMain;
-                if (t < tbest) {
-                    tbest = t;
-                    best = Plan{nc, P, L, 1};
+                const int rem = nc - (P - 1) * L;
+                if (L < 1 || rem < 1) continue;
+                const int lmax = rem > L ? rem : L;
+                // the rest in the last segment, or in the first (whose main
+                // pass needs no incoming state, but whose pre-pass everyone waits for)
+                const double t_last = L * kPre + kFlag1 + kScan + kFlag2 + lmax * kMain;
+                const double t_first =
+                    lmax * kPre + kFlag1 + kScan + std::max(rem * kMain, kFlag2 + L * kMain);
+                if (t_last < tbest) {
+                    tbest = t_last;
+                    best = Plan{nc, P, L, 1, 0};
+                }
+                // (row scans only: the column scans' pre-pass, on strided row
+                // slabs, is slower, and measured no gain)
+                if (pr.dir < 2 && t_first < tbest) {
+                    tbest = t_first;
+                    best = Plan{nc, P, L, 1, 1};
                 }
             }
         }
@@ -1182,7 +1204,7 @@ Plan make_plan(const Problem &pr) {
         const double t = waves * L * (kMain + kPre) + (P - 1) * kFold + kFlag;
         if (t < tbest) {
             tbest = t;
-            best = Plan{nc, P, L, 0};
+            best = Plan{nc, P, L, 0, 0};
         }
     }
     return best;
@@ -1236,7 +1258,14 @@ bool fused_supported(const Problem &pr) {
     return true;
 }
 
-size_t fused_workspace_bytes(const Problem &pr) { return ws_layout(pr, make_plan(pr)).total; }
+// The plan may differ between row and column scans; the workspace size covers
+// both, so a size queried without the direction fits every call.
+size_t fused_workspace_bytes(const Problem &pr) {
+    Problem rows = pr, cols = pr;
+    rows.dir = 0;
+    cols.dir = 2;
+    return std::max(ws_layout(rows, make_plan(rows)).total, ws_layout(cols, make_plan(cols)).total);
+}
 
 // One launch for the 64-wide sub-problem (key half kh, value half vh).
 static int launch_fused_part(const Problem &pr, const Plan &pl, const WsLayout &wl, void *ws,
@@ -1321,6 +1350,7 @@ static int launch_fused_part(const Problem &pr, const Plan &pl, const WsLayout &
     // launch guarantees it.  If this device holds fewer CTAs (a partitioned
     // GPU), the same plan runs with per-segment folds instead.
     p.coop = (pl.coop && coresident(func) >= (int)grid.x) ? 1 : 0;
+    p.rem_first = pl.rem_first;
     cudaLaunchConfig_t cfg;
     memset(&cfg, 0, sizeof(cfg));
     cfg.gridDim = grid;
