@@ -127,6 +127,9 @@ struct FusedParams {
     // boxes of `boxh` consecutive grid rows of one column (boxh: the largest
     // power of two <= 64 that divides grid_h, so no box crosses a column).
     CUtensorMap tm_q, tm_k, tm_v, tm_la;
+    // head sizes d_v = 128: the second value half's tile view (the launch's
+    // planes are (value half, b, h), value half slowest)
+    CUtensorMap tm_v2;
     const void *q, *k, *v;
     const float *la;
     void *out;
@@ -138,7 +141,10 @@ struct FusedParams {
     int *flag2;     // [BH*P] 1: this CTA's slice of every S_in is written (coop)
     unsigned *ctr;  // [0] ticket, [1] finished CTAs
     int *err;
-    int n, gh, gw, dir, nc, P, L, BH;
+    int n, gh, gw, dir, nc, P, L;
+    int BH;   // planes of this launch: BHt x nvh
+    int BHt;  // planes of the tensors (B H)
+    int nvh;  // value halves processed by this launch (1, or 2 when d_v = 128)
     // coop: every CTA is resident at once (cooperative launch) and the
     // boundary states come from the transposed scan; otherwise each segment
     // folds the earlier aggregates itself
@@ -338,7 +344,9 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
     tc_fence_after_sync();
     const uint32_t tbase = s_tmem;
     const int ticket = s_ticket;
-    const int bh = ticket / p.P, seg = ticket % p.P;
+    // launch plane bhf = (value half, tensor plane bh), segment seg
+    const int bhf = ticket / p.P, seg = ticket % p.P;
+    const int vpart = bhf / p.BHt, bh = bhf - vpart * p.BHt;
     // every segment has L chunks but one, which has the rest (possibly more):
     // the last, or with rem_first the first
     const int rem = p.nc - (p.P - 1) * p.L;
@@ -348,7 +356,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
     const int L = c_end - c_begin;
     const int npre = (seg < p.P - 1) ? L : 0;  // the last segment needs no aggregate
     const int n_items = npre + L;
-    const size_t slot = (size_t)bh * p.P + seg;
+    const size_t slot = (size_t)bhf * p.P + seg;
     constexpr uint32_t kFmt = BF16 ? 1u : 0u;
 
     if ((unsigned)ticket >= (unsigned)(p.BH * p.P)) {
@@ -365,6 +373,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
         const uint64_t pol_once = l2_policy_evict_first();
         bool ok = true;
         uint32_t issued = 0;  // bit s: the last use of stage s had its copies issued
+        const CUtensorMap *vmap = vpart ? &p.tm_v2 : &p.tm_v;
         for (int it = 0; it < n_items; ++it) {
             const int s = it % kStages;
             const bool pre = it < npre;
@@ -387,7 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
 #ifdef GTR_CHECKED
             {  // every box / gather of this chunk inside the tensor maps
                 const int p0 = (p.dir & 1) ? (p.n - FC - c * FC) : c * FC;
-                bool cok = bh < p.BH;
+                bool cok = bh < p.BHt && vpart < p.nvh;
                 if (p.dir < 2) {
                     cok = cok && p0 > -FC && p0 < p.n;
                 } else if (p.boxh == 0) {
@@ -425,7 +434,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
                 if (p.dir < 2) {
                     if (lane == 0) {
                         tma_load_3d_pol(st + ST_K, &p.tm_k, &bar_full[s], 0, p0, bh, pol);
-                        tma_load_3d_pol(st + ST_V, &p.tm_v, &bar_full[s], 0, p0, bh, pol);
+                        tma_load_3d_pol(st + ST_V, vmap, &bar_full[s], 0, p0, bh, pol);
                         tma_load_3d_pol(st + ST_LA, &p.tm_la, &bar_full[s], 0, p0, bh, pol);
                         if (!pre) tma_load_3d_pol(st + ST_Q, &p.tm_q, &bar_full[s], 0, p0, bh, pol_once);
                     }
@@ -439,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
                         }
                         const int m = 4 * lane;
                         tma_gather4_pol(st + ST_K + m * 128, &p.tm_k, &bar_full[s], 0, r[0], r[1], r[2], r[3], pol);
-                        tma_gather4_pol(st + ST_V + m * 128, &p.tm_v, &bar_full[s], 0, r[0], r[1], r[2], r[3], pol);
+                        tma_gather4_pol(st + ST_V + m * 128, vmap, &bar_full[s], 0, r[0], r[1], r[2], r[3], pol);
                         tma_gather4_pol(st + ST_LA + m * 256, &p.tm_la, &bar_full[s], 0, r[0], r[1], r[2], r[3], pol);
                         if (!pre)
                             tma_gather4_pol(st + ST_Q + m * 128, &p.tm_q, &bar_full[s], 0, r[0], r[1], r[2], r[3],
@@ -452,7 +461,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
                         const int x = pp >= 0 ? pp / p.gh : -1, y = pp >= 0 ? pp % p.gh : 0;
                         const int r = bx * h;
                         tma_load_4d_pol(st + ST_K + r * 128, &p.tm_k, &bar_full[s], 0, x, y, bh, pol);
-                        tma_load_4d_pol(st + ST_V + r * 128, &p.tm_v, &bar_full[s], 0, x, y, bh, pol);
+                        tma_load_4d_pol(st + ST_V + r * 128, vmap, &bar_full[s], 0, x, y, bh, pol);
                         tma_load_4d_pol(st + ST_LA + r * 256, &p.tm_la, &bar_full[s], 0, x, y, bh, pol);
                         if (!pre)
                             tma_load_4d_pol(st + ST_Q + r * 128, &p.tm_q, &bar_full[s], 0, x, y, bh, pol_once);
@@ -790,7 +799,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
             if (warp == kWarpEpi0) {
                 bool got = true;
                 for (int j = lane; j < p.P - 1; j += 32)
-                    got = wait_flag(p.flag + kWsFlagStride * ((size_t)bh * p.P + j)) && got;
+                    got = wait_flag(p.flag + kWsFlagStride * ((size_t)bhf * p.P + j)) && got;
                 if (!__all_sync(0xffffffffu, got) && lane == 0) {
                     s_abort = 1;
                     latch_error(p.err, kDevErrTimeout);
@@ -801,19 +810,19 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
             // stage this CTA's slice of every aggregate (A buffers, unused until
             // the first mask) and the plane's gate totals, every load in
             // flight at once, then scan the slice's pairs through the segments
-            const float2 *agp = reinterpret_cast<const float2 *>(p.agg + (size_t)bh * p.P * 4096);
-            float2 *sinp = reinterpret_cast<float2 *>(p.sin + (size_t)bh * p.P * 4096);
+            const float2 *agp = reinterpret_cast<const float2 *>(p.agg + (size_t)bhf * p.P * 4096);
+            float2 *sinp = reinterpret_cast<float2 *>(p.sin + (size_t)bhf * p.P * 4096);
             float2 *sA = reinterpret_cast<float2 *>(sm + OFF_A);
             float *sG = reinterpret_cast<float *>(sm + OFF_SCAN);
             const int u0 = seg * 2048 / p.P, u1 = (seg + 1) * 2048 / p.P;
             const int m = u1 - u0, nA = (p.P - 1) * m;
-            if (ok && !index_ok(bh < p.BH && seg < p.P && p.P <= kMaxScanSegments && u1 <= 2048, p.err)) ok = false;
+            if (ok && !index_ok(bhf < p.BH && seg < p.P && p.P <= kMaxScanSegments && u1 <= 2048, p.err)) ok = false;
             if (ok) {
                 float gt[8];  // (P - 1) * 64 <= 8 * kEpiThreads gate totals
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     const int e = et + j * kEpiThreads;
-                    if (e < (p.P - 1) * 64) gt[j] = __ldcg(p.aggg + (size_t)bh * p.P * 64 + e);
+                    if (e < (p.P - 1) * 64) gt[j] = __ldcg(p.aggg + (size_t)bhf * p.P * 64 + e);
                 }
                 for (int e0 = et; e0 < nA; e0 += 8 * kEpiThreads) {  // one pass: nA <= 8 * kEpiThreads
                     float2 t[8];
@@ -849,7 +858,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
                 if (warp == kWarpEpi0) {
                     bool got = true;
                     for (int j = lane; j < p.P; j += 32)
-                        got = wait_flag(p.flag2 + kWsFlagStride * ((size_t)bh * p.P + j)) && got;
+                        got = wait_flag(p.flag2 + kWsFlagStride * ((size_t)bhf * p.P + j)) && got;
                     if (!__all_sync(0xffffffffu, got) && lane == 0) {
                         s_abort = 1;
                         latch_error(p.err, kDevErrTimeout);
@@ -871,7 +880,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
         } else if (seg > 0) {  // fold the earlier segments' aggregates, nearest first
             if (warp == kWarpEpi0) {
                 bool got = true;
-                for (int j = lane; j < seg; j += 32) got = wait_flag(p.flag + kWsFlagStride * ((size_t)bh * p.P + j)) && got;
+                for (int j = lane; j < seg; j += 32) got = wait_flag(p.flag + kWsFlagStride * ((size_t)bhf * p.P + j)) && got;
                 if (!__all_sync(0xffffffffu, got) && lane == 0) {
                     s_abort = 1;
                     latch_error(p.err, kDevErrTimeout);
@@ -882,10 +891,10 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
             // The earlier segments' gate totals, copied once (coalesced) into
             // the A buffers, which stay unused until the first mask.
             float *sGt = reinterpret_cast<float *>(sm + OFF_A);
-            if (ok && !index_ok(bh < p.BH && seg < p.P && seg <= kMaxSegments, p.err)) ok = false;
+            if (ok && !index_ok(bhf < p.BH && seg < p.P && seg <= kMaxSegments, p.err)) ok = false;
             if (ok)
                 for (int e = tid - 32 * kWarpEpi0; e < seg * 64; e += kEpiThreads)
-                    sGt[e] = __ldcg(p.aggg + (size_t)bh * p.P * 64 + e);
+                    sGt[e] = __ldcg(p.aggg + (size_t)bhf * p.P * 64 + e);
             named_bar_sync(kBarEpi, kEpiThreads);
             float2 acc[4];  // log-gate sums of the segments between the source and this one
 #pragma unroll
@@ -894,7 +903,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
             // in flight while one is folded (same summation order as a plain loop)
             float2 vb[kFoldDepth][8];
             auto load = [&](int d, float2 *vv) {
-                const float *ag = p.agg + ((size_t)bh * p.P + (seg - 1 - d)) * 4096;
+                const float *ag = p.agg + ((size_t)bhf * p.P + (seg - 1 - d)) * 4096;
 #pragma unroll
                 for (int x = 0; x < 16; x += 2) {
                     const int j = r0 + 8 * ((x >> 1) & 1), i = hc + 8 * (x >> 2) + cq;
@@ -970,7 +979,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
                 for (int h = 0; h < 2; ++h) {
                     const size_t raster = (size_t)(prow[h] - bh * p.n);
                     yoff[h] = ((t_img * p.n + raster) * p.H + t_head) * 64 + hc + cq;
-                    if (r0 + 8 * h < plen && index_ok(yoff[h] + 26 <= (size_t)p.BH * p.n * 64, p.err)) {
+                    if (r0 + 8 * h < plen && index_ok(yoff[h] + 26 <= (size_t)p.BHt * p.n * 64, p.err)) {
                         const uint32_t *zp = reinterpret_cast<const uint32_t *>(reinterpret_cast<const T *>(p.z) +
                                                                                 yoff[h]);
 #pragma unroll
@@ -1004,7 +1013,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
                     const int row = r0 + 8 * h;
                     const float ss = sTail[(kp & 1) * 128 + row] + sTail[(kp & 1) * 128 + 64 + row];
                     const float rs = rsqrtf(fmaf(ss, 1.f / 64.f, p.eps));
-                    if (ok && row < plen && index_ok(yoff[h] + 26 <= (size_t)p.BH * p.n * 64, p.err)) {
+                    if (ok && row < plen && index_ok(yoff[h] + 26 <= (size_t)p.BHt * p.n * 64, p.err)) {
                         uint32_t *yp = reinterpret_cast<uint32_t *>(reinterpret_cast<T *>(p.y) + yoff[h]);
 #pragma unroll
                         for (int c = 0; c < 4; ++c) {
@@ -1023,9 +1032,9 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
                 // slower than the extra store instructions.)
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    if (r0 + 8 * h < plen && index_ok(prow[h] >= 0 && prow[h] < p.BH * p.n, p.err)) {
+                    if (r0 + 8 * h < plen && index_ok(prow[h] >= 0 && prow[h] < p.BHt * p.n, p.err)) {
                         uint32_t *dst = reinterpret_cast<uint32_t *>(reinterpret_cast<T *>(p.out) +
-                                                                     (size_t)prow[h] * p.ldo + hc + cq);
+                                                                     (size_t)prow[h] * p.ldo + 64 * vpart + hc + cq);
                         if (p.acc_out) {  // second key half: add to the first half's output
 #pragma unroll
                             for (int c = 0; c < 4; ++c) {
@@ -1109,8 +1118,8 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fused_kernel(const __grid_con
             plen = len;
         }
         if (L > 0) emit(L - 1);
-        if (seg == p.P - 1 && p.final_state && ok && index_ok(bh < p.BH, p.err)) {
-            float *fs = p.final_state + (size_t)bh * p.fs_bh;
+        if (seg == p.P - 1 && p.final_state && ok && index_ok(bhf < p.BH, p.err)) {
+            float *fs = p.final_state + (size_t)bh * p.fs_bh + 64 * vpart;
 #pragma unroll
             for (int x = 0; x < 16; ++x) {
                 const int j = r0 + 8 * ((x >> 1) & 1), i = hc + 8 * (x >> 2) + cq + (x & 1);
@@ -1163,12 +1172,16 @@ struct Plan {
 // on B200 (microseconds): a main-pass chunk, a pre-pass chunk, one folded
 // aggregate, the transposed scan, and the fixed cost of publishing and
 // waiting for flags.
+// Planes of one launch: every (b, h), twice when d_v = 128 (both value halves
+// of a key half in one launch).
+int launch_planes(const Problem &pr) { return pr.B * pr.H * (pr.dv / FD); }
+
 Plan make_plan(const Problem &pr) {
     // kFlag: publishing and the flag round of the fold; the cooperative plans
     // split it into the aggregates' round (kFlag1) and the scan's (kFlag2)
     constexpr double kMain = 2.2, kPre = 1.2, kFold = 0.5, kFlag = 3.0, kScan = 3.0, kFlag1 = 2.0, kFlag2 = 1.8;
     const int nc = (pr.n + FC - 1) / FC;
-    const int bh = pr.B * pr.H;
+    const int bh = launch_planes(pr);
     Plan best{nc, 1, nc, 0, 0};
     double tbest = nc * kMain * (double)((bh + kSMs - 1) / kSMs);
     const int pmax = nc < kMaxSegments ? nc : kMaxSegments;
@@ -1218,7 +1231,7 @@ struct WsLayout {
 // second half); the segment states after it.
 WsLayout ws_layout(const Problem &pr, const Plan &pl) {
     auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
-    const size_t slots = pl.P > 1 ? (size_t)pr.B * pr.H * pl.P : 0;
+    const size_t slots = pl.P > 1 ? (size_t)launch_planes(pr) * pl.P : 0;
     WsLayout w;
     w.ctr = 0;
     w.flag = 256;
@@ -1267,9 +1280,10 @@ size_t fused_workspace_bytes(const Problem &pr) {
     return std::max(ws_layout(rows, make_plan(rows)).total, ws_layout(cols, make_plan(cols)).total);
 }
 
-// One launch for the 64-wide sub-problem (key half kh, value half vh).
+// One launch for key half kh and every value half (its planes are (value
+// half, b, h)).
 static int launch_fused_part(const Problem &pr, const Plan &pl, const WsLayout &wl, void *ws,
-                             int kh, int vh, cudaStream_t st) {
+                             int kh, cudaStream_t st) {
     FusedParams p;
     memset(&p, 0, sizeof(p));
     char *w = static_cast<char *>(ws);
@@ -1305,8 +1319,10 @@ static int launch_fused_part(const Problem &pr, const Plan &pl, const WsLayout &
         const uint32_t box[4] = {FD, 1, (uint32_t)boxh, 1};
         return encode_tile_map(m, base, dt, 4, dims, str, box, sw);
     };
+    const int nvh = pr.dv / FD;
     if (enc(&p.tm_q, pr.q, pr.dk, FD * kh, dt16, 2, false) || enc(&p.tm_k, pr.k, pr.dk, FD * kh, dt16, 2, false) ||
-        enc(&p.tm_v, pr.v, pr.dv, FD * vh, dt16, 2, true) ||
+        enc(&p.tm_v, pr.v, pr.dv, 0, dt16, 2, true) ||
+        enc(&p.tm_v2, pr.v, pr.dv, FD * (nvh - 1), dt16, 2, true) ||
         enc(&p.tm_la, pr.la, pr.dk, FD * kh, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, false))
         return GTR_GLA_ERR_CUDA;
     p.boxh = boxh;
@@ -1314,10 +1330,10 @@ static int launch_fused_part(const Problem &pr, const Plan &pl, const WsLayout &
     p.k = pr.k;
     p.v = pr.v;
     p.la = pr.la;
-    p.out = static_cast<char *>(pr.out) + (size_t)FD * vh * 2;
+    p.out = pr.out;  // the kernel adds 64 columns per value half
     p.ldo = pr.dv;
     p.acc_out = kh > 0;
-    p.final_state = pr.final_state ? pr.final_state + (size_t)FD * kh * pr.dv + FD * vh : nullptr;
+    p.final_state = pr.final_state ? pr.final_state + (size_t)FD * kh * pr.dv : nullptr;
     p.fs_bh = pr.dk * pr.dv;
     p.fs_ld = pr.dv;
     p.agg = reinterpret_cast<float *>(w + wl.agg);
@@ -1334,7 +1350,9 @@ static int launch_fused_part(const Problem &pr, const Plan &pl, const WsLayout &
     p.nc = pl.nc;
     p.P = pl.P;
     p.L = pl.L;
-    p.BH = pr.B * pr.H;
+    p.BHt = pr.B * pr.H;
+    p.nvh = nvh;
+    p.BH = p.BHt * nvh;
     const dim3 grid(p.BH * p.P);
     p.z = pr.z;
     p.wn = pr.wn;
@@ -1368,18 +1386,18 @@ static int launch_fused_part(const Problem &pr, const Plan &pl, const WsLayout &
     return cudaPeekAtLastError() == cudaSuccess ? GTR_GLA_OK : GTR_GLA_ERR_CUDA;
 }
 
-// Head sizes of 128 run as 64-wide sub-problems, one launch each, in stream
-// order: first every value half of key half 0 (which writes the output),
-// then key half 1 (which adds to it).  The launches share the workspace; each
-// leaves its header zeroed for the next.
+// Head sizes of 128 run as 64-wide sub-problems: one launch per key half, in
+// stream order, each covering both value halves when d_v = 128 (its planes
+// are (value half, b, h)): key half 0 writes the output, key half 1 adds to
+// it.  The launches share the workspace; each leaves its header zeroed for
+// the next.
 int launch_fused(const Problem &pr, void *ws, cudaStream_t st) {
     const Plan pl = make_plan(pr);
     const WsLayout wl = ws_layout(pr, pl);
-    for (int kh = 0; kh < pr.dk / FD; ++kh)
-        for (int vh = 0; vh < pr.dv / FD; ++vh) {
-            const int rc = launch_fused_part(pr, pl, wl, ws, kh, vh, st);
-            if (rc != GTR_GLA_OK) return rc;
-        }
+    for (int kh = 0; kh < pr.dk / FD; ++kh) {
+        const int rc = launch_fused_part(pr, pl, wl, ws, kh, st);
+        if (rc != GTR_GLA_OK) return rc;
+    }
     return GTR_GLA_OK;
 }
 
