@@ -109,7 +109,7 @@ int gtr_gla_fwd(const void *q, const void *k, const void *v, const float *log_al
  *              GTR_GLA_ERR_CHUNK).  The result does not depend on it
  *              beyond rounding.  F16/BF16 with chunk 64 run the fused
  *              tensor-core kernel (head sizes of 128 as 64-wide parts, one
- *              launch each); every other combination runs the three-phase
+ *              launch per key half); every other combination runs the three-phase
  *              CUDA-core path.
  *   workspace: device buffer of at least gtr_gla_workspace_size(...) bytes,
  *              256-byte aligned, zero-filled before its first use.  Every call

@@ -5,21 +5,25 @@
 // Dense Prediction" (x-techcon article, section 算子) -- chunks compute their
 // own state contribution in parallel, boundary states are passed along, each
 // chunk's output is produced in parallel, scores stay on chip -- mapped onto
-// one launch of 576-thread CTAs, one per SM (head sizes of 128 run as four
-// launches of 64-wide parts, see launch_fused):
+// one launch of 576-thread CTAs, one per SM (head sizes of 128 run as one
+// launch per 64-wide key half, both value halves in it, see launch_fused):
 //
-//   * a CTA owns a segment of L consecutive 64-token chunks of one (b,h);
-//     CTAs take their segment from a ticket counter, so a segment only ever
-//     waits for segments that were started before it;
+//   * a CTA owns a segment of consecutive 64-token chunks of one (b,h); when
+//     the CTAs may run in several waves they take their segment from a
+//     ticket counter, so a segment only ever waits for segments that were
+//     started before it; one-wave plans run as a cooperative launch;
 //   * pre-pass (every segment but the last of its (b,h)): the segment's
 //     aggregate state contribution, transposed,
 //       A_seg^T = sum_c V_c^T (k_c . e^{G_after(c) + g_c - b_c}),
 //     accumulates in TMEM (chunks visited last to first, every factor <= 1)
 //     and is published with the segment's gate totals (one release store of
 //     a flag with a cache line of its own);
-//   * boundary: the incoming state is the fold of every earlier segment's
-//     aggregate, nearest first, S_in = sum_j diag(e^{G(j..seg)}) A_j (a fixed
-//     order: results are bitwise reproducible);
+//   * boundary: the incoming state S_in = sum_j diag(e^{G(j..seg)}) A_j over
+//     the earlier segments' aggregates, by a transposed scan across the
+//     plane's CTAs (cooperative launches: each CTA scans a slice of the state
+//     elements through all segments) or by each segment folding the earlier
+//     aggregates, nearest first (a fixed order either way: results are
+//     bitwise reproducible);
 //   * main pass, chunk by chunk:
 //       scores = Q^ K~^T        (tf32 MMA; Q^ = q . e^{b}, K~ = k . e^{-b},
 //                                b: in-chunk inclusive log-gate sums)
@@ -155,10 +159,10 @@ struct FusedParams {
     int rem_first;
     // Head sizes of 128 run as 64-wide sub-problems (every key row of the
     // state evolves on its own and every value column too; the output is
-    // the sum over the key halves): `out` and `final_state` point at the
-    // sub-problem's corner, ldo is the output row stride in elements,
-    // acc_out adds to what is already in `out`, fs_bh / fs_ld are the final
-    // state's (b,h) and row strides.
+    // the sum over the key halves): `out` is the output, `final_state` the
+    // key half's first row of it (each value half adds 64 columns), ldo the
+    // output row stride in elements, acc_out adds to what is already in
+    // `out`, fs_bh / fs_ld the final state's (b,h) and row strides.
     int ldo, acc_out, fs_bh, fs_ld;
     int boxh;  // rows per box (64 for row scans); 0: four-row gathers (column
                // scans whose grid_h is not a multiple of 8, where a box of V

@@ -55,7 +55,7 @@ int encode_tile_map_sw(CUtensorMap *m, const void *base, CUtensorMapDataType dt,
                        int swizzle_bytes);
 
 // Single-kernel tensor-core path (gla_fused.cu): fp16/bf16, chunk 64, d_k and d_v
-// each 64 or 128 (head sizes of 128 as one launch per 64-wide part).
+// each 64 or 128 (head sizes of 128 as one launch per 64-wide key half).
 bool fused_supported(const Problem &p);
 size_t fused_workspace_bytes(const Problem &p);
 int launch_fused(const Problem &p, void *ws, cudaStream_t st);

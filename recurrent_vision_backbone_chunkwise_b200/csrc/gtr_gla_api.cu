@@ -111,8 +111,8 @@ static int validate(const Problem &p) {
 }
 
 // fp16/bf16 with chunk 64 run the fused tensor-core kernel (head sizes of 128
-// as 64-wide parts); everything else (fp32 I/O, other chunk lengths) the
-// three-phase CUDA-core path.
+// as one launch per 64-wide key half); everything else (fp32 I/O, other chunk
+// lengths) the three-phase CUDA-core path.
 static size_t workspace_bytes(const Problem &p) {
     return fused_supported(p) ? fused_workspace_bytes(p) : generic_workspace_bytes(p);
 }
