@@ -110,3 +110,28 @@ def test_fused_tail(lib, direction):
     assert lib.gtr_gla_status(vp(st)) == 0
     o_ref, _ = oracle.forward(q, k, v, la, direction)
     assert rel(y, otail.forward(o_ref, z, w, 1e-5)) <= 5e-3
+
+
+def _random_cases(n=24, seed=2024):
+    import random
+
+    rng = random.Random(seed)
+    cases = []
+    for _ in range(n):
+        d_k, d_v = rng.choice([(64, 64), (64, 64), (64, 64), (128, 128), (64, 128), (128, 64)])
+        dtype = rng.choice(["f16", "f16", "bf16"])
+        chunk = 64 if rng.random() < 0.8 else rng.choice([32, 128 if d_k == 64 else 32])
+        if chunk != 64:
+            dtype = rng.choice(["f16", "f32"])
+        cases.append((Shape(rng.randint(1, 4), rng.randint(1, 16), rng.randint(1, 48), rng.randint(1, 48), d_k, d_v),
+                      dtype, rng.randint(0, 3), chunk))
+    return cases
+
+
+@pytest.mark.parametrize("shape,dtype,direction,chunk", _random_cases())
+def test_random_shapes(lib, shape, dtype, direction, chunk):
+    """Seeded random batches, head counts, grids, head sizes, directions,
+    dtypes and chunk lengths: the plan's segment counts and lengths, the
+    cooperative and folding boundary paths and both places of the leftover
+    chunks all come up; every index check passes and the result matches."""
+    run(lib, shape, dtype, direction, chunk=chunk, seed=shape.B * 7 + shape.grid_h)
