@@ -21,14 +21,19 @@
 //   6. per plane: the totals of the later chunks, exclusive    (bwd_carry)
 //   7. per token: dlog_alpha += the carry of its chunk           (bwd_add_carry)
 // Tokens are addressed in place through scan_to_raster, as in the forward pass.
+// The in-chunk log-gate sums b are kept in the log2 domain and every gate
+// factor (all <= 1) is one hardware 2^x (relative error about 2^-22).
 #include "../../include/gtr_gla_bwd.h"
+#include "sm100.cuh"
 #include "gla_common.cuh"
 #include "gla_internal.h"
 
 namespace gtr {
 namespace {
 
+using sm100::fast_exp2;
 constexpr int kT = 256;
+constexpr float kLog2e = 1.4426950408889634f;
 
 template <typename T, int DK, int DV, int C>
 __global__ void __launch_bounds__(kT) bwd_chunk_state(const T *__restrict__ k, const T *__restrict__ v,
@@ -58,15 +63,15 @@ __global__ void __launch_bounds__(kT) bwd_chunk_state(const T *__restrict__ k, c
     for (int i = threadIdx.x; i < DK; i += kT) {  // prefix sums per key dimension
         float acc = 0.f;
         for (int u = 0; u < C; ++u) {
-            acc += b[u * DK + i];
+            acc = fmaf(b[u * DK + i], kLog2e, acc);  // log2 domain
             b[u * DK + i] = acc;
         }
-        gam[((size_t)bh * nc + c) * DK + i] = expf(acc);
+        gam[((size_t)bh * nc + c) * DK + i] = fast_exp2(acc);
     }
     __syncthreads();
     for (int e = threadIdx.x; e < C * DK; e += kT) {
         const int u = e / DK, i = e % DK;
-        kh[e] = u < len ? kh[e] * expf(b[(C - 1) * DK + i] - b[e]) : 0.f;
+        kh[e] = u < len ? kh[e] * fast_exp2(b[(C - 1) * DK + i] - b[e]) : 0.f;
     }
     __syncthreads();
     for (int e = threadIdx.x; e < DK * DV; e += kT) {
@@ -121,12 +126,12 @@ __global__ void __launch_bounds__(kT) bwd_chunk_dstate(const T *__restrict__ q, 
     for (int i = threadIdx.x; i < DK; i += kT) {
         float acc = 0.f;
         for (int u = 0; u < C; ++u) {
-            acc += b[u * DK + i];
+            acc = fmaf(b[u * DK + i], kLog2e, acc);  // log2 domain
             b[u * DK + i] = acc;
         }
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < C * DK; e += kT) qh[e] *= expf(b[e]);
+    for (int e = threadIdx.x; e < C * DK; e += kT) qh[e] *= fast_exp2(b[e]);
     __syncthreads();
     for (int e = threadIdx.x; e < DK * DV; e += kT) {
         const int i = e / DV, j = e % DV;
@@ -160,19 +165,26 @@ __global__ void __launch_bounds__(kT) bwd_chunk_grads(
     const T *__restrict__ dO, const float *__restrict__ S_in, const float *__restrict__ dS_out,
     const float *__restrict__ dS_final, const float *__restrict__ S_final, T *__restrict__ dq, T *__restrict__ dk,
     T *__restrict__ dv, float *__restrict__ dla, float *__restrict__ tot, int n, int gh, int gw, int dir, int nc) {
+    // Rows padded by one float (DKP, DVP): the loops below walk a column with
+    // consecutive lanes on consecutive rows, which padding keeps free of
+    // shared-memory bank conflicts.  The chunk's S_in and dS_out are staged
+    // the same way (their rows are read across lanes too).
+    constexpr int DKP = DK + 1, DVP = DV + 1;
     extern __shared__ float sm[];
-    float *b = sm;             // [C][DK]
-    float *qs = b + C * DK;    // [C][DK]
-    float *ks = qs + C * DK;   // [C][DK]
-    float *vs = ks + C * DK;   // [C][DV]
-    float *gs = vs + C * DV;   // [C][DV]  dO
-    float *W = gs + C * DV;    // [C][C]   dO_t . v_s, s <= t
-    float *A = W + C * C;      // [C][C]   scores, s <= t
-    float *db = A + C * C;     // [C][DK]
+    float *b = sm;              // [C][DKP]  in-chunk log2-gate sums
+    float *qs = b + C * DKP;    // [C][DKP]
+    float *ks = qs + C * DKP;   // [C][DKP]
+    float *vs = ks + C * DKP;   // [C][DVP]
+    float *gs = vs + C * DVP;   // [C][DVP]  dO
+    float *W = gs + C * DVP;    // [C][C]    dO_t . v_s, s <= t
+    float *A = W + C * C;       // [C][C]    scores, s <= t
+    float *db = A + C * C;      // [C][DK]
+    float *Si = db + C * DK;    // [DK][DVP] S_in of the chunk
+    float *Do = Si + DK * DVP;  // [DK][DVP] dS_out of the chunk
     const int c = blockIdx.x, bh = blockIdx.y, t0 = c * C, len = min(C, n - t0);
     const size_t pk = (size_t)bh * n * DK, pv = (size_t)bh * n * DV;
-    const float *Si = S_in + ((size_t)bh * nc + c) * DK * DV;
-    const float *Do = dS_out + ((size_t)bh * nc + c) * DK * DV;
+    const float *Sig = S_in + ((size_t)bh * nc + c) * DK * DV;
+    const float *Dog = dS_out + ((size_t)bh * nc + c) * DK * DV;
     for (int e = threadIdx.x; e < C * DK; e += kT) {
         const int u = e / DK, i = e % DK;
         float lv = 0.f, qv = 0.f, kv = 0.f;
@@ -182,9 +194,9 @@ __global__ void __launch_bounds__(kT) bwd_chunk_grads(
             qv = to_f32(q[pk + r * DK + i]);
             kv = to_f32(k[pk + r * DK + i]);
         }
-        b[e] = lv;
-        qs[e] = qv;
-        ks[e] = kv;
+        b[u * DKP + i] = lv;
+        qs[u * DKP + i] = qv;
+        ks[u * DKP + i] = kv;
     }
     for (int e = threadIdx.x; e < C * DV; e += kT) {
         const int u = e / DV, j = e % DV;
@@ -194,15 +206,20 @@ __global__ void __launch_bounds__(kT) bwd_chunk_grads(
             vv = to_f32(v[pv + r * DV + j]);
             gv = to_f32(dO[pv + r * DV + j]);
         }
-        vs[e] = vv;
-        gs[e] = gv;
+        vs[u * DVP + j] = vv;
+        gs[u * DVP + j] = gv;
+    }
+    for (int e = threadIdx.x; e < DK * DV; e += kT) {
+        const int i = e / DV, j = e % DV;
+        Si[i * DVP + j] = Sig[e];
+        Do[i * DVP + j] = Dog[e];
     }
     __syncthreads();
     for (int i = threadIdx.x; i < DK; i += kT) {
         float acc = 0.f;
         for (int u = 0; u < C; ++u) {
-            acc += b[u * DK + i];
-            b[u * DK + i] = acc;
+            acc = fmaf(b[u * DKP + i], kLog2e, acc);  // log2 domain
+            b[u * DKP + i] = acc;
         }
     }
     __syncthreads();
@@ -210,34 +227,34 @@ __global__ void __launch_bounds__(kT) bwd_chunk_grads(
         const int t = e / C, s = e % C;
         float w = 0.f, a = 0.f;
         if (s <= t && t < len) {
-            for (int j = 0; j < DV; ++j) w = fmaf(gs[t * DV + j], vs[s * DV + j], w);
+            for (int j = 0; j < DV; ++j) w = fmaf(gs[t * DVP + j], vs[s * DVP + j], w);
             for (int i = 0; i < DK; ++i)
-                a = fmaf(qs[t * DK + i] * ks[s * DK + i], expf(b[t * DK + i] - b[s * DK + i]), a);
+                a = fmaf(qs[t * DKP + i] * ks[s * DKP + i], fast_exp2(b[t * DKP + i] - b[s * DKP + i]), a);
         }
         W[e] = w;
         A[e] = a;
     }
     __syncthreads();
-    const float *gend = b + (C - 1) * DK;  // g: the chunk's total (padded tokens add log 1 = 0)
+    const float *gend = b + (C - 1) * DKP;  // g: the chunk's total (padded tokens add log 1 = 0)
     for (int e = threadIdx.x; e < C * DK; e += kT) {  // dq and dk, one (token, key dim) per step
         const int t = e / DK, i = e % DK;
         float gq = 0.f, gk = 0.f;
         if (t < len) {
             float inter = 0.f, intra = 0.f;
-            for (int j = 0; j < DV; ++j) inter = fmaf(gs[t * DV + j], Si[i * DV + j], inter);
+            for (int j = 0; j < DV; ++j) inter = fmaf(gs[t * DVP + j], Si[i * DVP + j], inter);
             for (int s = 0; s <= t; ++s)
-                intra = fmaf(W[t * C + s] * ks[s * DK + i], expf(b[t * DK + i] - b[s * DK + i]), intra);
-            gq = expf(b[t * DK + i]) * inter + intra;
+                intra = fmaf(W[t * C + s] * ks[s * DKP + i], fast_exp2(b[t * DKP + i] - b[s * DKP + i]), intra);
+            gq = fast_exp2(b[t * DKP + i]) * inter + intra;
             float st = 0.f, kk = 0.f;  // token t as the key side s
             for (int u = t; u < len; ++u)
-                kk = fmaf(W[u * C + t] * qs[u * DK + i], expf(b[u * DK + i] - b[t * DK + i]), kk);
-            for (int j = 0; j < DV; ++j) st = fmaf(vs[t * DV + j], Do[i * DV + j], st);
-            gk = kk + expf(gend[i] - b[t * DK + i]) * st;
+                kk = fmaf(W[u * C + t] * qs[u * DKP + i], fast_exp2(b[u * DKP + i] - b[t * DKP + i]), kk);
+            for (int j = 0; j < DV; ++j) st = fmaf(vs[t * DVP + j], Do[i * DVP + j], st);
+            gk = kk + fast_exp2(gend[i] - b[t * DKP + i]) * st;
             const size_t r = (size_t)scan_to_raster(t0 + t, n, gh, gw, dir);
             dq[pk + r * DK + i] = from_f32<T>(gq);
             dk[pk + r * DK + i] = from_f32<T>(gk);
         }
-        db[e] = qs[e] * gq - ks[e] * gk;
+        db[e] = qs[t * DKP + i] * gq - ks[t * DKP + i] * gk;
         if (t0 + t == n - 1 && dS_final) {  // the scan's last token: the final state's gate
             float f = 0.f;
             for (int j = 0; j < DV; ++j)
@@ -249,8 +266,9 @@ __global__ void __launch_bounds__(kT) bwd_chunk_grads(
         const int s = e / DV, j = e % DV;
         if (s >= len) continue;
         float acc = 0.f;
-        for (int t = s; t < len; ++t) acc = fmaf(A[t * C + s], gs[t * DV + j], acc);
-        for (int i = 0; i < DK; ++i) acc = fmaf(ks[s * DK + i] * expf(gend[i] - b[s * DK + i]), Do[i * DV + j], acc);
+        for (int t = s; t < len; ++t) acc = fmaf(A[t * C + s], gs[t * DVP + j], acc);
+        for (int i = 0; i < DK; ++i)
+            acc = fmaf(ks[s * DKP + i] * fast_exp2(gend[i] - b[s * DKP + i]), Do[i * DVP + j], acc);
         const size_t r = (size_t)scan_to_raster(t0 + s, n, gh, gw, dir);
         dv[pv + r * DV + j] = from_f32<T>(acc);
     }
@@ -320,7 +338,7 @@ int launch_bwd(const T *q, const T *k, const T *v, const float *la, const T *dO,
     float *Sf = reinterpret_cast<float *>(w + l.Sf);
     const dim3 gchunk(nc, BH);
     const size_t sm1 = (size_t)(2 * C * DK + C * DV) * 4;
-    const size_t sm5 = (size_t)(4 * C * DK + 2 * C * DV + 2 * C * C) * 4;
+    const size_t sm5 = (size_t)(3 * C * (DK + 1) + 2 * C * (DV + 1) + 2 * C * C + C * DK + 2 * DK * (DV + 1)) * 4;
     int rc;
     if ((rc = ensure_smem((const void *)bwd_chunk_state<T, DK, DV, C>, sm1))) return rc;
     if ((rc = ensure_smem((const void *)bwd_chunk_dstate<T, DK, DV, C>, sm1))) return rc;
