@@ -33,6 +33,9 @@ namespace {
 
 using sm100::fast_exp2;
 constexpr int kT = 256;
+// bwd_chunk_grads holds one CTA per SM (its shared memory), so it runs 32
+// warps to hide the latency of its shared-memory loads.
+constexpr int kTG = 1024;
 constexpr float kLog2e = 1.4426950408889634f;
 
 template <typename T, int DK, int DV, int C>
@@ -160,7 +163,7 @@ __global__ void bwd_dstate_scan(float *__restrict__ Z, const float *__restrict__
 // Per chunk: dq, dk, dv in the I/O dtype at raster positions; dlog_alpha gets
 // the in-chunk suffix sums of db (fp32), the chunk total goes to tot.
 template <typename T, int DK, int DV, int C>
-__global__ void __launch_bounds__(kT) bwd_chunk_grads(
+__global__ void __launch_bounds__(kTG) bwd_chunk_grads(
     const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v, const float *__restrict__ la,
     const T *__restrict__ dO, const float *__restrict__ S_in, const float *__restrict__ dS_out,
     const float *__restrict__ dS_final, const float *__restrict__ S_final, T *__restrict__ dq, T *__restrict__ dk,
@@ -185,7 +188,7 @@ __global__ void __launch_bounds__(kT) bwd_chunk_grads(
     const size_t pk = (size_t)bh * n * DK, pv = (size_t)bh * n * DV;
     const float *Sig = S_in + ((size_t)bh * nc + c) * DK * DV;
     const float *Dog = dS_out + ((size_t)bh * nc + c) * DK * DV;
-    for (int e = threadIdx.x; e < C * DK; e += kT) {
+    for (int e = threadIdx.x; e < C * DK; e += kTG) {
         const int u = e / DK, i = e % DK;
         float lv = 0.f, qv = 0.f, kv = 0.f;
         if (u < len) {
@@ -198,7 +201,7 @@ __global__ void __launch_bounds__(kT) bwd_chunk_grads(
         qs[u * DKP + i] = qv;
         ks[u * DKP + i] = kv;
     }
-    for (int e = threadIdx.x; e < C * DV; e += kT) {
+    for (int e = threadIdx.x; e < C * DV; e += kTG) {
         const int u = e / DV, j = e % DV;
         float vv = 0.f, gv = 0.f;
         if (u < len) {
@@ -209,13 +212,13 @@ __global__ void __launch_bounds__(kT) bwd_chunk_grads(
         vs[u * DVP + j] = vv;
         gs[u * DVP + j] = gv;
     }
-    for (int e = threadIdx.x; e < DK * DV; e += kT) {
+    for (int e = threadIdx.x; e < DK * DV; e += kTG) {
         const int i = e / DV, j = e % DV;
         Si[i * DVP + j] = Sig[e];
         Do[i * DVP + j] = Dog[e];
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < DK; i += kT) {
+    for (int i = threadIdx.x; i < DK; i += kTG) {
         float acc = 0.f;
         for (int u = 0; u < C; ++u) {
             acc = fmaf(b[u * DKP + i], kLog2e, acc);  // log2 domain
@@ -223,7 +226,7 @@ __global__ void __launch_bounds__(kT) bwd_chunk_grads(
         }
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < C * C; e += kT) {  // W and A, pair by pair
+    for (int e = threadIdx.x; e < C * C; e += kTG) {  // W and A, pair by pair
         const int t = e / C, s = e % C;
         float w = 0.f, a = 0.f;
         if (s <= t && t < len) {
@@ -236,7 +239,7 @@ __global__ void __launch_bounds__(kT) bwd_chunk_grads(
     }
     __syncthreads();
     const float *gend = b + (C - 1) * DKP;  // g: the chunk's total (padded tokens add log 1 = 0)
-    for (int e = threadIdx.x; e < C * DK; e += kT) {  // dq and dk, one (token, key dim) per step
+    for (int e = threadIdx.x; e < C * DK; e += kTG) {  // dq and dk, one (token, key dim) per step
         const int t = e / DK, i = e % DK;
         float gq = 0.f, gk = 0.f;
         if (t < len) {
@@ -262,7 +265,7 @@ __global__ void __launch_bounds__(kT) bwd_chunk_grads(
             db[e] += f;
         }
     }
-    for (int e = threadIdx.x; e < C * DV; e += kT) {  // dv
+    for (int e = threadIdx.x; e < C * DV; e += kTG) {  // dv
         const int s = e / DV, j = e % DV;
         if (s >= len) continue;
         float acc = 0.f;
@@ -273,7 +276,7 @@ __global__ void __launch_bounds__(kT) bwd_chunk_grads(
         dv[pv + r * DV + j] = from_f32<T>(acc);
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < DK; i += kT) {  // suffix sums of db inside the chunk
+    for (int i = threadIdx.x; i < DK; i += kTG) {  // suffix sums of db inside the chunk
         float acc = 0.f;
         for (int u = len - 1; u >= 0; --u) {
             acc += db[u * DK + i];
@@ -347,7 +350,7 @@ int launch_bwd(const T *q, const T *k, const T *v, const float *la, const T *dO,
     bwd_state_scan<DK, DV><<<dim3((DK * DV + 255) / 256, BH), 256, 0, st>>>(S, gam, Sf, nc);
     bwd_chunk_dstate<T, DK, DV, C><<<gchunk, kT, sm1, st>>>(q, dO, la, Z, n, gh, gw, dir, nc);
     bwd_dstate_scan<DK, DV><<<dim3((DK * DV + 255) / 256, BH), 256, 0, st>>>(Z, gam, dSf, nc);
-    bwd_chunk_grads<T, DK, DV, C><<<gchunk, kT, sm5, st>>>(q, k, v, la, dO, S, Z, dSf, Sf, dq, dk, dv, dla, tot, n,
+    bwd_chunk_grads<T, DK, DV, C><<<gchunk, kTG, sm5, st>>>(q, k, v, la, dO, S, Z, dSf, Sf, dq, dk, dv, dla, tot, n,
                                                              gh, gw, dir, nc);
     bwd_carry<DK><<<dim3((DK + 63) / 64, BH), 64, 0, st>>>(tot, nc);
     const long long total = (long long)BH * n * DK;
