@@ -32,14 +32,17 @@ namespace gtr {
 namespace {
 
 using sm100::fast_exp2;
-constexpr int kT = 256;
-// bwd_chunk_grads holds one CTA per SM (its shared memory), so it runs 32
-// warps to hide the latency of its shared-memory loads.
-constexpr int kTG = 1024;
+// bwd_chunk_grads holds one CTA per SM (its shared memory) and runs 32 warps
+// to hide the latency of its shared-memory loads.  The two other chunk
+// kernels (48 KB each) take the thread count NT: 1024 when the problem gives
+// about one CTA per SM, else 256, so that four CTAs share an SM and overlap
+// each other's serial prefix-sum phase.
+constexpr int kT = 1024;
+constexpr int kTSmall = 256;
 constexpr float kLog2e = 1.4426950408889634f;
 
-template <typename T, int DK, int DV, int C>
-__global__ void __launch_bounds__(kT) bwd_chunk_state(const T *__restrict__ k, const T *__restrict__ v,
+template <typename T, int DK, int DV, int C, int NT>
+__global__ void __launch_bounds__(NT) bwd_chunk_state(const T *__restrict__ k, const T *__restrict__ v,
                                                       const float *__restrict__ la, float *__restrict__ dS,
                                                       float *__restrict__ gam, int n, int gh, int gw, int dir,
                                                       int nc) {
@@ -47,7 +50,7 @@ __global__ void __launch_bounds__(kT) bwd_chunk_state(const T *__restrict__ k, c
     float *b = sm, *kh = b + C * DK, *vs = kh + C * DK;
     const int c = blockIdx.x, bh = blockIdx.y, t0 = c * C, len = min(C, n - t0);
     const size_t pk = (size_t)bh * n * DK, pv = (size_t)bh * n * DV;
-    for (int e = threadIdx.x; e < C * DK; e += kT) {
+    for (int e = threadIdx.x; e < C * DK; e += NT) {
         const int u = e / DK, i = e % DK;
         float lv = 0.f, kv = 0.f;
         if (u < len) {
@@ -58,12 +61,12 @@ __global__ void __launch_bounds__(kT) bwd_chunk_state(const T *__restrict__ k, c
         b[e] = lv;
         kh[e] = kv;
     }
-    for (int e = threadIdx.x; e < C * DV; e += kT) {
+    for (int e = threadIdx.x; e < C * DV; e += NT) {
         const int u = e / DV, j = e % DV;
         vs[e] = u < len ? to_f32(v[pv + (size_t)scan_to_raster(t0 + u, n, gh, gw, dir) * DV + j]) : 0.f;
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < DK; i += kT) {  // prefix sums per key dimension
+    for (int i = threadIdx.x; i < DK; i += NT) {  // prefix sums per key dimension
         float acc = 0.f;
         for (int u = 0; u < C; ++u) {
             acc = fmaf(b[u * DK + i], kLog2e, acc);  // log2 domain
@@ -72,12 +75,12 @@ __global__ void __launch_bounds__(kT) bwd_chunk_state(const T *__restrict__ k, c
         gam[((size_t)bh * nc + c) * DK + i] = fast_exp2(acc);
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < C * DK; e += kT) {
+    for (int e = threadIdx.x; e < C * DK; e += NT) {
         const int u = e / DK, i = e % DK;
         kh[e] = u < len ? kh[e] * fast_exp2(b[(C - 1) * DK + i] - b[e]) : 0.f;
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < DK * DV; e += kT) {
+    for (int e = threadIdx.x; e < DK * DV; e += NT) {
         const int i = e / DV, j = e % DV;
         float acc = 0.f;
         for (int u = 0; u < len; ++u) acc = fmaf(kh[u * DK + i], vs[u * DV + j], acc);
@@ -93,6 +96,7 @@ __global__ void bwd_state_scan(float *__restrict__ dS, const float *__restrict__
     if (e >= DK * DV) return;
     const int i = e / DV;
     float s = 0.f;
+#pragma unroll 4
     for (int c = 0; c < nc; ++c) {
         float *p = dS + ((size_t)bh * nc + c) * DK * DV + e;
         const float d = *p;
@@ -102,15 +106,15 @@ __global__ void bwd_state_scan(float *__restrict__ dS, const float *__restrict__
     S_final[(size_t)bh * DK * DV + e] = s;
 }
 
-template <typename T, int DK, int DV, int C>
-__global__ void __launch_bounds__(kT) bwd_chunk_dstate(const T *__restrict__ q, const T *__restrict__ dO,
+template <typename T, int DK, int DV, int C, int NT>
+__global__ void __launch_bounds__(NT) bwd_chunk_dstate(const T *__restrict__ q, const T *__restrict__ dO,
                                                        const float *__restrict__ la, float *__restrict__ Z, int n,
                                                        int gh, int gw, int dir, int nc) {
     extern __shared__ float sm[];
     float *b = sm, *qh = b + C * DK, *gs = qh + C * DK;
     const int c = blockIdx.x, bh = blockIdx.y, t0 = c * C, len = min(C, n - t0);
     const size_t pk = (size_t)bh * n * DK, pv = (size_t)bh * n * DV;
-    for (int e = threadIdx.x; e < C * DK; e += kT) {
+    for (int e = threadIdx.x; e < C * DK; e += NT) {
         const int u = e / DK, i = e % DK;
         float lv = 0.f, qv = 0.f;
         if (u < len) {
@@ -121,12 +125,12 @@ __global__ void __launch_bounds__(kT) bwd_chunk_dstate(const T *__restrict__ q, 
         b[e] = lv;
         qh[e] = qv;
     }
-    for (int e = threadIdx.x; e < C * DV; e += kT) {
+    for (int e = threadIdx.x; e < C * DV; e += NT) {
         const int u = e / DV, j = e % DV;
         gs[e] = u < len ? to_f32(dO[pv + (size_t)scan_to_raster(t0 + u, n, gh, gw, dir) * DV + j]) : 0.f;
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < DK; i += kT) {
+    for (int i = threadIdx.x; i < DK; i += NT) {
         float acc = 0.f;
         for (int u = 0; u < C; ++u) {
             acc = fmaf(b[u * DK + i], kLog2e, acc);  // log2 domain
@@ -134,9 +138,9 @@ __global__ void __launch_bounds__(kT) bwd_chunk_dstate(const T *__restrict__ q, 
         }
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < C * DK; e += kT) qh[e] *= fast_exp2(b[e]);
+    for (int e = threadIdx.x; e < C * DK; e += NT) qh[e] *= fast_exp2(b[e]);
     __syncthreads();
-    for (int e = threadIdx.x; e < DK * DV; e += kT) {
+    for (int e = threadIdx.x; e < DK * DV; e += NT) {
         const int i = e / DV, j = e % DV;
         float acc = 0.f;
         for (int u = 0; u < len; ++u) acc = fmaf(qh[u * DK + i], gs[u * DV + j], acc);
@@ -152,6 +156,7 @@ __global__ void bwd_dstate_scan(float *__restrict__ Z, const float *__restrict__
     if (e >= DK * DV) return;
     const int i = e / DV;
     float cur = dS_final ? dS_final[(size_t)bh * DK * DV + e] : 0.f;
+#pragma unroll 4
     for (int c = nc - 1; c >= 0; --c) {
         float *p = Z + ((size_t)bh * nc + c) * DK * DV + e;
         const float z = *p;
@@ -163,7 +168,7 @@ __global__ void bwd_dstate_scan(float *__restrict__ Z, const float *__restrict__
 // Per chunk: dq, dk, dv in the I/O dtype at raster positions; dlog_alpha gets
 // the in-chunk suffix sums of db (fp32), the chunk total goes to tot.
 template <typename T, int DK, int DV, int C>
-__global__ void __launch_bounds__(kTG) bwd_chunk_grads(
+__global__ void __launch_bounds__(kT) bwd_chunk_grads(
     const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v, const float *__restrict__ la,
     const T *__restrict__ dO, const float *__restrict__ S_in, const float *__restrict__ dS_out,
     const float *__restrict__ dS_final, const float *__restrict__ S_final, T *__restrict__ dq, T *__restrict__ dk,
@@ -188,7 +193,7 @@ __global__ void __launch_bounds__(kTG) bwd_chunk_grads(
     const size_t pk = (size_t)bh * n * DK, pv = (size_t)bh * n * DV;
     const float *Sig = S_in + ((size_t)bh * nc + c) * DK * DV;
     const float *Dog = dS_out + ((size_t)bh * nc + c) * DK * DV;
-    for (int e = threadIdx.x; e < C * DK; e += kTG) {
+    for (int e = threadIdx.x; e < C * DK; e += kT) {
         const int u = e / DK, i = e % DK;
         float lv = 0.f, qv = 0.f, kv = 0.f;
         if (u < len) {
@@ -201,7 +206,7 @@ __global__ void __launch_bounds__(kTG) bwd_chunk_grads(
         qs[u * DKP + i] = qv;
         ks[u * DKP + i] = kv;
     }
-    for (int e = threadIdx.x; e < C * DV; e += kTG) {
+    for (int e = threadIdx.x; e < C * DV; e += kT) {
         const int u = e / DV, j = e % DV;
         float vv = 0.f, gv = 0.f;
         if (u < len) {
@@ -212,13 +217,13 @@ __global__ void __launch_bounds__(kTG) bwd_chunk_grads(
         vs[u * DVP + j] = vv;
         gs[u * DVP + j] = gv;
     }
-    for (int e = threadIdx.x; e < DK * DV; e += kTG) {
+    for (int e = threadIdx.x; e < DK * DV; e += kT) {
         const int i = e / DV, j = e % DV;
         Si[i * DVP + j] = Sig[e];
         Do[i * DVP + j] = Dog[e];
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < DK; i += kTG) {
+    for (int i = threadIdx.x; i < DK; i += kT) {
         float acc = 0.f;
         for (int u = 0; u < C; ++u) {
             acc = fmaf(b[u * DKP + i], kLog2e, acc);  // log2 domain
@@ -226,7 +231,7 @@ __global__ void __launch_bounds__(kTG) bwd_chunk_grads(
         }
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < C * C; e += kTG) {  // W and A, pair by pair
+    for (int e = threadIdx.x; e < C * C; e += kT) {  // W and A, pair by pair
         const int t = e / C, s = e % C;
         float w = 0.f, a = 0.f;
         if (s <= t && t < len) {
@@ -239,7 +244,7 @@ __global__ void __launch_bounds__(kTG) bwd_chunk_grads(
     }
     __syncthreads();
     const float *gend = b + (C - 1) * DKP;  // g: the chunk's total (padded tokens add log 1 = 0)
-    for (int e = threadIdx.x; e < C * DK; e += kTG) {  // dq and dk, one (token, key dim) per step
+    for (int e = threadIdx.x; e < C * DK; e += kT) {  // dq and dk, one (token, key dim) per step
         const int t = e / DK, i = e % DK;
         float gq = 0.f, gk = 0.f;
         if (t < len) {
@@ -265,7 +270,7 @@ __global__ void __launch_bounds__(kTG) bwd_chunk_grads(
             db[e] += f;
         }
     }
-    for (int e = threadIdx.x; e < C * DV; e += kTG) {  // dv
+    for (int e = threadIdx.x; e < C * DV; e += kT) {  // dv
         const int s = e / DV, j = e % DV;
         if (s >= len) continue;
         float acc = 0.f;
@@ -276,7 +281,7 @@ __global__ void __launch_bounds__(kTG) bwd_chunk_grads(
         dv[pv + r * DV + j] = from_f32<T>(acc);
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < DK; i += kTG) {  // suffix sums of db inside the chunk
+    for (int i = threadIdx.x; i < DK; i += kT) {  // suffix sums of db inside the chunk
         float acc = 0.f;
         for (int u = len - 1; u >= 0; --u) {
             acc += db[u * DK + i];
@@ -342,15 +347,24 @@ int launch_bwd(const T *q, const T *k, const T *v, const float *la, const T *dO,
     const dim3 gchunk(nc, BH);
     const size_t sm1 = (size_t)(2 * C * DK + C * DV) * 4;
     const size_t sm5 = (size_t)(3 * C * (DK + 1) + 2 * C * (DV + 1) + 2 * C * C + C * DK + 2 * DK * (DV + 1)) * 4;
+    const bool wide = (long long)nc * BH <= 2 * 148;  // about one chunk CTA per SM
     int rc;
-    if ((rc = ensure_smem((const void *)bwd_chunk_state<T, DK, DV, C>, sm1))) return rc;
-    if ((rc = ensure_smem((const void *)bwd_chunk_dstate<T, DK, DV, C>, sm1))) return rc;
+    if ((rc = ensure_smem((const void *)bwd_chunk_state<T, DK, DV, C, kT>, sm1))) return rc;
+    if ((rc = ensure_smem((const void *)bwd_chunk_state<T, DK, DV, C, kTSmall>, sm1))) return rc;
+    if ((rc = ensure_smem((const void *)bwd_chunk_dstate<T, DK, DV, C, kT>, sm1))) return rc;
+    if ((rc = ensure_smem((const void *)bwd_chunk_dstate<T, DK, DV, C, kTSmall>, sm1))) return rc;
     if ((rc = ensure_smem((const void *)bwd_chunk_grads<T, DK, DV, C>, sm5))) return rc;
-    bwd_chunk_state<T, DK, DV, C><<<gchunk, kT, sm1, st>>>(k, v, la, S, gam, n, gh, gw, dir, nc);
+    if (wide)
+        bwd_chunk_state<T, DK, DV, C, kT><<<gchunk, kT, sm1, st>>>(k, v, la, S, gam, n, gh, gw, dir, nc);
+    else
+        bwd_chunk_state<T, DK, DV, C, kTSmall><<<gchunk, kTSmall, sm1, st>>>(k, v, la, S, gam, n, gh, gw, dir, nc);
     bwd_state_scan<DK, DV><<<dim3((DK * DV + 255) / 256, BH), 256, 0, st>>>(S, gam, Sf, nc);
-    bwd_chunk_dstate<T, DK, DV, C><<<gchunk, kT, sm1, st>>>(q, dO, la, Z, n, gh, gw, dir, nc);
+    if (wide)
+        bwd_chunk_dstate<T, DK, DV, C, kT><<<gchunk, kT, sm1, st>>>(q, dO, la, Z, n, gh, gw, dir, nc);
+    else
+        bwd_chunk_dstate<T, DK, DV, C, kTSmall><<<gchunk, kTSmall, sm1, st>>>(q, dO, la, Z, n, gh, gw, dir, nc);
     bwd_dstate_scan<DK, DV><<<dim3((DK * DV + 255) / 256, BH), 256, 0, st>>>(Z, gam, dSf, nc);
-    bwd_chunk_grads<T, DK, DV, C><<<gchunk, kTG, sm5, st>>>(q, k, v, la, dO, S, Z, dSf, Sf, dq, dk, dv, dla, tot, n,
+    bwd_chunk_grads<T, DK, DV, C><<<gchunk, kT, sm5, st>>>(q, k, v, la, dO, S, Z, dSf, Sf, dq, dk, dv, dla, tot, n,
                                                              gh, gw, dir, nc);
     bwd_carry<DK><<<dim3((DK + 63) / 64, BH), 64, 0, st>>>(tot, nc);
     const long long total = (long long)BH * n * DK;

@@ -60,6 +60,7 @@ def test_backward_matches_oracle(direction, dtype):
     (Shape(1, 1, 1, 1, 64, 64), "f32", 1),    # one token
     (Shape(1, 6, 40, 40, 64, 64), "f16", 3),  # the 640x640 detection grid
     (Shape(1, 2, 16, 16, 64, 64), "bf16", 0),
+    (Shape(4, 12, 24, 24, 64, 64), "f16", 1),  # 432 chunk CTAs: the 256-thread chunk kernels
 ])
 def test_backward_edge_cases(shape, dtype, direction):
     run(shape, dtype, direction, with_final=True, seed=7)
