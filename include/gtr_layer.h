@@ -41,7 +41,9 @@
  * C not a positive multiple of 64 or above 2048, F <= 0 or not a multiple of
  * 8, too many tokens, n_layers < 1), _DIRECTION, _DTYPE, _ALIGN (a pointer not
  * 16-byte aligned), _WORKSPACE (NULL, too small or not 256-byte aligned),
- * _CUDA (a launch failed).
+ * _ALIAS (x, the bytes of the workspace the call uses and the weights do not
+ * all stay apart; weights may share memory among themselves), _CUDA (a
+ * launch failed).
  */
 #ifndef GTR_LAYER_H
 #define GTR_LAYER_H

@@ -253,6 +253,32 @@ int check_call(const void *x, int B, int gh, int gw, int C, int F, int dir, int 
     return GTR_GLA_OK;
 }
 
+bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
+    const char *pa = static_cast<const char *>(a), *pb = static_cast<const char *>(b);
+    return pa < pb + nb && pb < pa + na;
+}
+
+// x is updated in place and the workspace written, so neither may overlap
+// the other or any weight (weights may share memory among themselves).
+int check_alias(const void *x, const GtrLayerWeights *w, int B, int gh, int gw, int C, int F,
+                const void *workspace, const Layout &l) {
+    const size_t e = 2, M = (size_t)B * gh * gw, nx = M * C * e;
+    if (overlaps(x, nx, workspace, l.total)) return GTR_GLA_ERR_ALIAS;
+    const struct {
+        const void *p;
+        size_t n;
+    } wts[] = {{w->ln1_w, (size_t)C * 4},          {w->ln1_b, (size_t)C * 4},
+               {w->w_proj, (size_t)5 * C * C * e}, {w->b_a, (size_t)C * 4},
+               {w->w_n, (size_t)C * 4},            {w->w_o, (size_t)C * C * e},
+               {w->ln2_w, (size_t)C * 4},          {w->ln2_b, (size_t)C * 4},
+               {w->w_gu, (size_t)2 * F * C * e},   {w->b_gu, (size_t)2 * F * 4},
+               {w->w_dw, (size_t)9 * F * 4},       {w->b_dw, (size_t)F * 4},
+               {w->w_down, (size_t)C * F * e},     {w->b_down, (size_t)C * 4}};
+    for (const auto &t : wts)
+        if (overlaps(t.p, t.n, x, nx) || overlaps(t.p, t.n, workspace, l.total)) return GTR_GLA_ERR_ALIAS;
+    return GTR_GLA_OK;
+}
+
 int run_layer(void *x, const GtrLayerWeights *w, int B, int gh, int gw, int C, int F, int dir, int dtype,
               void *workspace, const Layout &l, cudaStream_t st) {
     char *ws = static_cast<char *>(workspace);
@@ -271,6 +297,7 @@ extern "C" int gtr_layer_fwd(void *x, const GtrLayerWeights *w, int B, int grid_
     if (rc) return rc;
     Layout l;
     if ((rc = check_call(x, B, grid_h, grid_w, C, F, direction, dtype, workspace, workspace_bytes, &l))) return rc;
+    if ((rc = check_alias(x, w, B, grid_h, grid_w, C, F, workspace, l))) return rc;
     return run_layer(x, w, B, grid_h, grid_w, C, F, direction, dtype, workspace, l, stream);
 }
 
@@ -284,6 +311,8 @@ extern "C" int gtr_backbone_fwd(void *x, const GtrLayerWeights *layers, int n_la
         if ((rc = check_weights(&layers[i]))) return rc;
     Layout l;
     if ((rc = check_call(x, B, grid_h, grid_w, C, F, 0, dtype, workspace, workspace_bytes, &l))) return rc;
+    for (int i = 0; i < n_layers; ++i)
+        if ((rc = check_alias(x, &layers[i], B, grid_h, grid_w, C, F, workspace, l))) return rc;
     for (int i = 0; i < n_layers; ++i)
         if ((rc = run_layer(x, &layers[i], B, grid_h, grid_w, C, F, i % 4, dtype, workspace, l, stream))) return rc;
     return GTR_GLA_OK;

@@ -249,6 +249,8 @@ def test_layer_workspace_size(gla):
     (dict(C=100), -2), (dict(C=4096), -2), (dict(F=0), -2), (dict(F=12), -2), (dict(B=0), -2),
     (dict(dir=4), -4), (dict(dtype=2), -6), (dict(x=0x20000008), -5), ("w_gu_misaligned", -5),
     (dict(ws=0), -8), (dict(wsb=1024), -8), (dict(ws=0x30000010), -8),
+    (dict(x=0x30000000), -11),            # x inside the workspace
+    ("w_o_on_x", -11), ("w_dw_in_ws", -11),
 ])
 def test_layer_argument_errors(gla, kw, code):
     from recurrent_vision_backbone_chunkwise_b200 import layer
@@ -257,7 +259,12 @@ def test_layer_argument_errors(gla, kw, code):
         kw = dict(w=_layer_struct(layer, w_o=0))
     elif kw == "w_gu_misaligned":
         kw = dict(w=_layer_struct(layer, w_gu=0x50000004))
+    elif kw == "w_o_on_x":
+        kw = dict(w=_layer_struct(layer, w_o=0x20000000 - 4096))  # [C, C] fp16 runs into x
+    elif kw == "w_dw_in_ws":
+        kw = dict(w=_layer_struct(layer, w_dw=0x30000100))
     assert call_layer(gla, **kw) == code
+
 
 
 def test_backbone_argument_errors(gla):
@@ -270,6 +277,8 @@ def test_backbone_argument_errors(gla):
     assert f(vp(0x20000000), None, 2, 1, 6, 7, 128, 512, gla.F16, vp(0x30000000), 1 << 34, None) == -1
     assert f(vp(0x20000000), arr, 0, 1, 6, 7, 128, 512, gla.F16, vp(0x30000000), 1 << 34, None) == -2
     assert f(vp(0x20000000), arr, 1, 1, 6, 7, 128, 512, gla.F16, vp(0x30000000), 1024, None) == -8
+    arr2 = (layer.GtrLayerWeights * 2)(_layer_struct(layer), _layer_struct(layer, b_down=0x20000000))
+    assert f(vp(0x20000000), arr2, 2, 1, 6, 7, 128, 512, gla.F16, vp(0x30000000), 1 << 34, None) == -11
 
 
 # ------------------------------------------------------------ fused output tail
