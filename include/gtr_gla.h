@@ -73,7 +73,8 @@ enum {
     GTR_GLA_ERR_WORKSPACE = -8,   /* workspace NULL or smaller than required      */
     GTR_GLA_ERR_CUDA = -9,        /* a CUDA runtime call or launch failed         */
     GTR_GLA_ERR_TIMEOUT = -10,    /* a device-side wait gave up (gtr_gla_status)  */
-    GTR_GLA_ERR_ALIAS = -11,      /* out overlaps an input                        */
+    GTR_GLA_ERR_ALIAS = -11,      /* out overlaps an input, or a caller workspace
+                                     overlaps a tensor argument                   */
     GTR_GLA_ERR_WORKSPACE_STATE = -12 /* a call found the workspace header not zero
                                          (calls sharing a workspace overlapped, or it
                                          was not zero-filled); reported by
@@ -115,7 +116,8 @@ int gtr_gla_fwd(const void *q, const void *k, const void *v, const float *log_al
  *              256-byte aligned, zero-filled before its first use.  Every call
  *              leaves it ready for the next one.  Calls that share a workspace
  *              must not overlap on the GPU.  May be NULL only when the
- *              required size is 0.
+ *              required size is 0.  The bytes it uses must not overlap q, k,
+ *              v, log_alpha, out or final_state (GTR_GLA_ERR_ALIAS).
  */
 int gtr_gla_fwd_ex(const void *q, const void *k, const void *v, const float *log_alpha,
                    void *out, float *final_state, int B, int H, int grid_h, int grid_w,
@@ -166,7 +168,8 @@ int gtr_gla_fwd_noalloc(const void *q, const void *k, const void *v, const float
  *              launch (gtr_output_tail_fwd).
  * Other arguments, errors and final_state as gtr_gla_fwd_ex; in addition
  * GTR_GLA_ERR_NULL for a NULL z or w_n, _SHAPE for eps < 0 or not finite,
- * _ALIGN for z or w_n, _ALIAS when y overlaps z, w_n or the workspace.
+ * _ALIGN for z or w_n, _ALIAS when y overlaps z or w_n, or the workspace
+ * overlaps any tensor argument.
  */
 int gtr_gla_fwd_tail(const void *q, const void *k, const void *v, const float *log_alpha,
                      const void *z, const float *w_n, float eps, void *y, float *final_state,

@@ -24,7 +24,7 @@
  * dtype GTR_GLA_F16, GTR_GLA_BF16 or GTR_GLA_F32; d_k = d_v = 64.  The
  * outputs must not overlap any input or each other.  workspace: at least
  * gtr_gla_bwd_workspace_size(...) bytes, 256-byte aligned (no zero-fill
- * needed).  Asynchronous and stream-ordered.
+ * needed), overlapping no tensor argument.  Asynchronous and stream-ordered.
  *
  * Errors (codes of gtr_gla.h, before anything is launched): GTR_GLA_ERR_NULL,
  * _SHAPE, _HEAD_DIM (d_k or d_v not 64), _DIRECTION, _ALIGN, _DTYPE,

@@ -445,6 +445,17 @@ extern "C" int gtr_gla_bwd(const void *q, const void *k, const void *v, const fl
     if (rc) return rc;
     const size_t need = gtr_gla_bwd_workspace_size(B, H, grid_h, grid_w, d_k, d_v);
     if (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 255u)) return GTR_GLA_ERR_WORKSPACE;
+    {  // the workspace is written: it may overlap no tensor argument
+        const size_t es = dtype == GTR_GLA_F32 ? 4 : 2, tok = (size_t)B * H * grid_h * grid_w;
+        const size_t nx = tok * 64 * es, nla = tok * 64 * 4, nfs = (size_t)B * H * 64 * 64 * 4;
+        const struct {
+            const void *p;
+            size_t n;
+        } t[] = {{q, nx},  {k, nx},  {v, nx},  {d_out, nx},         {dq, nx},
+                 {dk, nx}, {dv, nx}, {log_alpha, nla}, {dlog_alpha, nla}, {d_final_state, nfs}};
+        for (const auto &e : t)
+            if (overlaps(workspace, need, e.p, e.n)) return GTR_GLA_ERR_ALIAS;
+    }
     if (dtype == GTR_GLA_F16)
         return run_bwd<__half>(q, k, v, log_alpha, d_out, d_final_state, dq, dk, dv, dlog_alpha, B, H, grid_h, grid_w,
                                direction, workspace, stream);

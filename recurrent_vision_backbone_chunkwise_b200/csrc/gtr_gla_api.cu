@@ -110,6 +110,19 @@ static int validate(const Problem &p) {
     return GTR_GLA_OK;
 }
 
+// The workspace is written by the kernels, so its first `n` bytes may overlap
+// no tensor argument of the call (inputs, out or y, final_state).
+static bool workspace_touches(const Problem &p, const void *ws, size_t n) {
+    if (!ws || n == 0) return false;
+    const size_t es = elem_size(p.dtype);
+    const size_t tok = (size_t)p.B * p.H * p.n;
+    const size_t nq = tok * p.dk * es, nv = tok * p.dv * es, nla = tok * p.dk * 4;
+    const size_t nfs = (size_t)p.B * p.H * p.dk * p.dv * 4;
+    return overlaps(ws, n, p.q, nq) || overlaps(ws, n, p.k, nq) || overlaps(ws, n, p.v, nv) ||
+           overlaps(ws, n, p.la, nla) || overlaps(ws, n, p.out, nv) ||
+           (p.final_state && overlaps(ws, n, p.final_state, nfs));
+}
+
 // fp16/bf16 with chunk 64 run the fused tensor-core kernel (head sizes of 128
 // as one launch per 64-wide key half); everything else (fp32 I/O, other chunk
 // lengths) the three-phase CUDA-core path.
@@ -159,6 +172,7 @@ int gtr_gla_fwd_ex(const void *q, const void *k, const void *v, const float *log
     const size_t need = workspace_bytes(p);
     if (need > 0 && (!workspace || workspace_bytes_ < need || ((uintptr_t)workspace & 255u)))
         return GTR_GLA_ERR_WORKSPACE;
+    if (need > 0 && workspace_touches(p, workspace, need)) return GTR_GLA_ERR_ALIAS;
     int dev;
     if ((rc = current_device(&dev))) return rc;
     if ((rc = device_err_ptr(dev, &p.err))) return rc;
@@ -243,7 +257,9 @@ int gtr_gla_fwd_tail(const void *q, const void *k, const void *v, const float *l
     size_t obuf;
     const size_t need = tail_layout(p, &obuf);
     if (!workspace || workspace_bytes_ < need || ((uintptr_t)workspace & 255u)) return GTR_GLA_ERR_WORKSPACE;
-    if (overlaps(y, ny, workspace, need)) return GTR_GLA_ERR_ALIAS;
+    if (workspace_touches(p, workspace, need) || overlaps(z, ny, workspace, need) ||
+        overlaps(w_n, (size_t)p.H * p.dv * 4, workspace, need))
+        return GTR_GLA_ERR_ALIAS;
     int dev;
     if ((rc = current_device(&dev))) return rc;
     if ((rc = device_err_ptr(dev, &p.err))) return rc;

@@ -100,6 +100,7 @@ def call_ex(gla, **kw):
     (dict(chunk=48), -7), (dict(chunk=16), -7),
     (dict(ws=0), -8), (dict(wsb=16), -8), (dict(ws=WS + 16), -8),
     (dict(out=Q + 256), -11), (dict(fs=OUT), -11),
+    (dict(ws=OUT), -11), (dict(ws=LA + 4096), -11), (dict(ws=FS), -11),  # workspace on a tensor
 ])
 def test_argument_errors_return_before_launch(gla, kw, code):
     assert call_ex(gla, **kw) == code
@@ -299,6 +300,7 @@ def call_tail(gla, **kw):
     (dict(dk=48), -3), (dict(dir=5), -4), (dict(z=0x80000008), -5), (dict(w=0x90000004), -5),
     (dict(dtype=2), -6), (dict(wsb=0), -8), (dict(ws=0), -8),
     (dict(z=OUT + 64), -11), (dict(y=Q), -11), (dict(w=OUT + 256), -11),
+    (dict(ws=0x80000000), -11), (dict(ws=K), -11), (dict(ws=OUT), -11),  # workspace on z, k, y
 ])
 def test_tail_argument_errors(gla, kw, code):
     assert call_tail(gla, **kw) == code
@@ -344,6 +346,7 @@ def test_gemm_argument_errors(gla, kw, code):
     (dict(q=0), -1), (dict(dla=0), -1), (dict(B=0), -2), (dict(dk=128), -3), (dict(dir=4), -4),
     (dict(dq=Q + 8), -5), (dict(dtype=3), -6), (dict(ws=0), -8), (dict(wsb=16), -8),
     (dict(dq=K), -11), (dict(dv=0xA0000000 + 256), -11), (dict(dla=LA), -11),
+    (dict(ws=0xB0000000), -11), (dict(ws=FS), -11), (dict(ws=Q), -11),  # workspace on dk, dS_final, q
 ])
 def test_backward_argument_errors(gla, kw, code):
     a = dict(q=Q, k=K, v=V, la=LA, dO=OUT, dsf=FS, dq=0xA0000000, dk=0xB0000000, dv=0xC0000000,
