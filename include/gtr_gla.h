@@ -64,7 +64,9 @@ enum { GTR_GLA_F16 = 0, GTR_GLA_BF16 = 1, GTR_GLA_F32 = 2 };
 enum {
     GTR_GLA_OK = 0,
     GTR_GLA_ERR_NULL = -1,        /* a required pointer is NULL                   */
-    GTR_GLA_ERR_SHAPE = -2,       /* B, H, grid_h or grid_w <= 0, or too large    */
+    GTR_GLA_ERR_SHAPE = -2,       /* B, H, grid_h or grid_w <= 0, or too large:
+                                     B*H > 65535, grid_h*grid_w > 2^22 or
+                                     B*H*grid_h*grid_w >= 2^31                  */
     GTR_GLA_ERR_HEAD_DIM = -3,    /* (d_k, d_v) not supported                     */
     GTR_GLA_ERR_DIRECTION = -4,   /* direction not in [0, 3]                      */
     GTR_GLA_ERR_ALIGN = -5,       /* a pointer is not 16-byte aligned             */

@@ -80,6 +80,8 @@ static bool chunk_ok(int chunk, int dk) {
 static int validate_shape(int B, int H, int gh, int gw, int dk, int dv, int dtype, int chunk) {
     if (B <= 0 || H <= 0 || gh <= 0 || gw <= 0) return GTR_GLA_ERR_SHAPE;
     if ((long long)B * H > 65535 || (long long)gh * gw > (1LL << 22)) return GTR_GLA_ERR_SHAPE;
+    // token rows of all planes are 32-bit (row tables, TMA coordinates)
+    if ((long long)B * H * gh * gw >= (1LL << 31)) return GTR_GLA_ERR_SHAPE;
     if (dtype != GTR_GLA_F16 && dtype != GTR_GLA_BF16 && dtype != GTR_GLA_F32)
         return GTR_GLA_ERR_DTYPE;
     if (!head_dims_ok(dk, dv)) return GTR_GLA_ERR_HEAD_DIM;

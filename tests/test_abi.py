@@ -93,6 +93,7 @@ def call_ex(gla, **kw):
 @pytest.mark.parametrize("kw,code", [
     (dict(q=0), -1), (dict(la=0), -1), (dict(out=0), -1),
     (dict(B=0), -2), (dict(gh=-1), -2), (dict(H=70000), -2),
+    (dict(H=1024, gh=2048, gw=1024), -2),  # 2^31 token rows in all
     (dict(dk=32), -3), (dict(dv=96), -3),
     (dict(dir=4), -4), (dict(dir=-1), -4),
     (dict(q=Q + 8), -5), (dict(fs=FS + 4), -5),
