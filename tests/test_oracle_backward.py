@@ -1,6 +1,9 @@
 """Pins for the GLA gradient oracle (oracle/backward.py, gla_backward.c), CPU only.
 
 Each pin is independent of the oracle's code:
+- scalar examples worked by hand with the chain rule: three tokens in all
+  four directions (tests/golden/backward_scalar_1x3.json) and the two column
+  scans of a 2x2 grid (tests/golden/backward_scalar_2x2_columns.json);
 - central finite differences of the forward oracle (itself pinned in
   test_oracle_pins.py), as directional derivatives in all four directions and
   element by element on a tiny plane;
@@ -35,6 +38,36 @@ def _case(B=1, H=2, gh=3, gw=4, dk=3, dv=2, seed=0):
     dO = r.standard_normal((B, H, gh, gw, dv))
     dS = r.standard_normal((B, H, dk, dv))
     return q, k, v, la, dO, dS
+
+
+def _golden_scalar(name="backward_scalar_1x3.json"):
+    import json
+
+    with open(os.path.join(ROOT, "tests", "golden", name)) as f:
+        g = json.load(f)
+    shape = (1, 1, g["grid"][0], g["grid"][1], 1)
+    q, k, v = (np.array(g[n], dtype=np.float64).reshape(shape) for n in ("q", "k", "v"))
+    la = np.log(np.array(g["alpha"], dtype=np.float64)).reshape(shape)
+    dO = np.array(g["d_out"], dtype=np.float64).reshape(shape)
+    dS = np.full((1, 1, 1, 1), g["d_final_state"])
+    return g, (q, k, v, la, dO, dS)
+
+
+@pytest.mark.parametrize("name,direction", [("backward_scalar_1x3.json", d) for d in range(4)] +
+                         [("backward_scalar_2x2_columns.json", d) for d in (2, 3)])
+def test_hand_worked_scalar_gradients(name, direction):
+    g, (q, k, v, la, dO, dS) = _golden_scalar(name)
+    exp = next(e for e in g["expected"].values() if direction in e["directions"])
+    o, S = oracle.forward(q, k, v, la, direction)
+    assert np.allclose(o.ravel(), exp["out"], rtol=0, atol=1e-12)
+    assert abs(float(S.ravel()[0]) - exp["final_state"]) <= 1e-12
+    grads = ob.backward(q, k, v, la, dO, direction, d_final_state=dS)
+    for name, got in zip(("dq", "dk", "dv", "dlog_alpha"), grads):
+        assert np.allclose(np.asarray(got).ravel(), exp[name], rtol=0, atol=1e-12), name
+    # the chunked reorganisation at a chunk shorter than the scan
+    grads_c = ob.chunkwise_backward(q, k, v, la, dO, direction, chunk=2, d_final_state=dS)
+    for name, got in zip(("dq", "dk", "dv", "dlog_alpha"), grads_c):
+        assert np.allclose(np.asarray(got).ravel(), exp[name], rtol=0, atol=1e-12), name
 
 
 def _loss(q, k, v, la, dO, dS, direction):
@@ -160,6 +193,7 @@ def _run_pins(tmp, edit):
                     ignore=shutil.ignore_patterns("*.so", "__pycache__"))
     os.makedirs(os.path.join(tmp, "tests"))
     shutil.copy(os.path.abspath(__file__), os.path.join(tmp, "tests", "test_pins.py"))
+    shutil.copytree(os.path.join(ROOT, "tests", "golden"), os.path.join(tmp, "tests", "golden"))
     path = os.path.join(tmp, "oracle", "gla_backward.c")
     if edit:
         old, new = edit
