@@ -54,7 +54,8 @@ size_t gtr_swiglu_workspace_size(int B, int grid_h, int grid_w, int C, int F, in
  * gtr_swiglu_fwd -- y = Spatial SwiGLU(x) as above.
  *   dtype:     GTR_GLA_F16 or GTR_GLA_BF16 (else GTR_GLA_ERR_DTYPE).
  *   workspace: device buffer of at least gtr_swiglu_workspace_size(...)
- *              bytes, 256-byte aligned; calls sharing it must not overlap on
+ *              bytes, 256-byte aligned, overlapping no tensor argument
+ *              (GTR_GLA_ERR_ALIAS); calls sharing it must not overlap on
  *              the GPU.
  * Errors: GTR_GLA_ERR_NULL, _SHAPE (B, grid or C, F <= 0, or C, F not
  * multiples of 8), _DTYPE, _ALIGN, _ALIAS, _WORKSPACE, _CUDA; all but the

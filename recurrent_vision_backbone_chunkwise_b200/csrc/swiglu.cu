@@ -417,7 +417,12 @@ extern "C" int gtr_swiglu_fwd(const void *x, const void *w_gu, const float *b_gu
         return GTR_GLA_ERR_ALIAS;
     const SwLayout l = sw_layout(M, C, F, es);
     if (!workspace || workspace_bytes < l.total || ((uintptr_t)workspace & 255u)) return GTR_GLA_ERR_WORKSPACE;
-    if (overlap(y, ny, workspace, l.total)) return GTR_GLA_ERR_ALIAS;
+    if (overlap(workspace, l.total, y, ny) || overlap(workspace, l.total, x, ny) ||
+        overlap(workspace, l.total, w_gu, (size_t)2 * F * C * es) ||
+        overlap(workspace, l.total, w_down, (size_t)C * F * es) ||
+        overlap(workspace, l.total, b_gu, (size_t)2 * F * 4) || overlap(workspace, l.total, w_dw, (size_t)F * 36) ||
+        overlap(workspace, l.total, b_dw, (size_t)F * 4) || overlap(workspace, l.total, b_down, (size_t)C * 4))
+        return GTR_GLA_ERR_ALIAS;
     return swiglu_apply(x, w_gu, b_gu, w_dw, b_dw, w_down, b_down, nullptr, y, B, grid_h, grid_w, C, F, dtype,
                         workspace, stream);
 }

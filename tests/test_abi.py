@@ -146,6 +146,8 @@ def test_swiglu_argument_errors_before_launch(gla):
     q = [C.c_void_p((1 << 20) + (i << 32)) for i in range(8)]
     assert call(ptrs=q, ws=None) == -8                 # no workspace
     assert call(ptrs=q, wsb=16) == -8                  # workspace too small
+    assert call(ptrs=q) == -11                         # workspace on x
+    assert call(ptrs=q, ws=q[3]) == -11                # workspace on the depthwise taps
     assert swiglu.gtr_swiglu_workspace_size(1, 4, 4, 60, 256) == 0
     assert swiglu.gtr_swiglu_workspace_size(1, 40, 40, 384, 1536) > 1600 * 3 * 1536 * 2
 
